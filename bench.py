@@ -1,0 +1,399 @@
+"""Benchmark: SwiGLU MLP block (d=4096, ffn=14336, Llama-3.1-8B shapes) run
+through the direct-palette reconstructive GEMM on B200.
+
+One step = one forward pass of the block at a token batch: the gate GEMM,
+the up GEMM with SiLU(g)*u fused into its epilogue, and the down GEMM, all
+three reading compressed weights (sign+mantissa bytes, 4-bit palette indices,
+verbatim rows) and rebuilding BF16 on chip.  Synthetic N(0, 0.02) weights with
+1e-4 outliers x100 stand in for Llama-3.1-8B's MLP weights.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--batch B]
+    python bench.py --impl reference     # the CPU oracle on a bounded sample
+
+Prints one JSON line on rank 0.  Multi-GPU runs (torchrun) are independent
+replicas: the block does not shard on this path, so there is no collective in
+the data path; the timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "reconstructive MLP GEMM tokens/s & effective weight GB/s vs HBM roofline, B=1–256"
+D_MODEL, FFN = 4096, 14336
+SIGMA, OUTLIER_RATE, OUTLIER_SCALE, SEED = 0.02, 1e-4, 100.0, 2
+HBM_FALLBACK_GBS = 6650.0
+
+# DRAM traffic (read + write bytes) per launch of the direct-palette GEMM
+# kernel from ncu (see profiles/); None until a capture of the current kernel
+# exists.
+NCU_TRAFFIC_PER_LAUNCH = None
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return json.load(f), "measured"
+    except Exception:
+        return {"hbm_gbs": HBM_FALLBACK_GBS, "bf16_tflops": 1590.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms in the background."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return self
+
+        def reader():
+            for line in self.proc.stdout:
+                self.samples.append((time.time(), line.strip()))
+        self.thread = threading.Thread(target=reader, daemon=True)
+        self.thread.start()
+        return self
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        rows = []
+        for ts, line in self.samples:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            rows.append((ts, parts))
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        window = "timed region"
+        if not inside:
+            inside = rows
+            window = "whole run (timed region shorter than the 200 ms sampling interval)"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "window": "unavailable"}
+        sm = [float(p[1]) for _, p in inside if p[1].replace(".", "").isdigit()]
+        smax = [float(p[2]) for _, p in inside if p[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, p in inside for i in range(4) if p[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(inside), "window": window}
+
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl" if os.environ.get("UW_BENCH_BACKEND", "nccl") == "nccl" else "gloo",
+                                timeout=timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, v: float) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(world, v: float) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle leg (the reported CPU baseline and the --impl reference arm)
+# ---------------------------------------------------------------------------
+
+_ORACLE_PREP = {}
+
+
+def oracle_prepare(batch: int, row_fraction: float):
+    """Untimed preparation of the CPU sample: the first `row_fraction` of the
+    rows of gate, up and down in the direct-palette form (oracle encoder and
+    transcode), plus inputs of the right widths."""
+    key = (batch, row_fraction)
+    if key not in _ORACLE_PREP:
+        from mlp_huffman_coded_b200 import synth
+        from oracle import uw_oracle as O
+        mats = synth.mlp_block(D_MODEL, FFN, SIGMA, OUTLIER_RATE, OUTLIER_SCALE, SEED)
+        preps = []
+        for w in mats:
+            n = max(128, int(round(w.shape[0] * row_fraction / 128)) * 128)
+            enc = O.encode(np.ascontiguousarray(w[:n]))
+            preps.append((enc, O.transcode_palette(enc, lockstep=True), n / w.shape[0]))
+        xs = [synth.activations(batch, D_MODEL, 3), synth.activations(batch, D_MODEL, 3),
+              synth.activations(batch, FFN, 4)]
+        _ORACLE_PREP[key] = (preps, xs)
+    return _ORACLE_PREP[key]
+
+
+def oracle_block_sample(batch: int, row_fraction: float):
+    """Oracle work for one step on a row sample of each matrix: rebuild W from
+    the direct-palette form (sm + 4-bit indices + verbatim rows), float64
+    GEMM, SiLU(g) * u.  Returns the seconds scaled to the whole block."""
+    from oracle import uw_oracle as O
+    preps, xs = oracle_prepare(batch, row_fraction)
+    t0 = time.perf_counter()
+    outs = []
+    for (enc, idx4, _), x in zip(preps, xs):
+        outs.append(O.gemm(O.rebuild_from_idx4(enc, idx4), x))
+    _ = O.silu(outs[0]) * outs[1]
+    dt = time.perf_counter() - t0
+    frac = sum(f for _, _, f in preps) / 3
+    return dt / frac
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    from threadpoolctl import threadpool_limits
+    frac = args.ref_fraction
+    with threadpool_limits(limits=1):
+        oracle_prepare(args.batch, frac)
+        for _ in range(args.warmup):
+            oracle_block_sample(args.batch, frac)
+        times = [oracle_block_sample(args.batch, frac) for _ in range(args.steps)]
+    step_s = sum(times) / len(times)   # full-block seconds per step
+    value = args.batch / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(args),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{frac:.4f} of the rows of gate, up and down per step, scaled to the full block"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_dict(args):
+    return {"workload": f"SwiGLU MLP block d={D_MODEL} ffn={FFN} (Llama-3.1-8B shapes), direct-palette "
+                        f"reconstructive GEMM, batch {args.batch}",
+            "batch": args.batch, "d_model": D_MODEL, "ffn": FFN, "pipeline": "direct palette (gate, up, down)",
+            "weights": f"N(0,{SIGMA}) bf16, outliers {OUTLIER_RATE} x{OUTLIER_SCALE}, seed {SEED}",
+            "l2": "inputs larger than L2: 3 compressed matrices (~268 MB) streamed per step, L2 is 126 MB"}
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def run_gpu(args, world, rank, local):
+    import torch
+    from mlp_huffman_coded_b200 import synth, uw
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    B = args.batch
+    mats = synth.mlp_block(D_MODEL, FFN, SIGMA, OUTLIER_RATE, OUTLIER_SCALE, SEED)
+    encs = [uw.encode(w) for w in mats]
+    dms = []
+    ws0 = uw.Workspace(256, device=dev)
+    for e in encs:
+        dms.append(uw.DeviceMatrix(e, device=dev).prepare_direct_palette(ws0))
+    ws0.check("load-time transcode")
+    pipes = [uw.PIPE_DIRECT] * 3
+    ws = uw.Workspace(uw.mlp_workspace_bytes(*dms, pipes, B), device=dev)
+    x_host = synth.activations(B, D_MODEL, 3)
+    x = torch.from_numpy(x_host.view(np.int16)).to(dev)
+    y = torch.empty(B, D_MODEL, dtype=torch.int16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        uw.mlp_block(*dms, pipes, x, y, ws, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    ws.check("warmup")
+
+    sampler = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
+                           if os.environ.get("CUDA_VISIBLE_DEVICES", "").replace(",", "").isdigit() else local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    launches0 = uw.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    e1.synchronize()
+    t_wall1 = time.time()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    launches = uw.launch_count() - launches0
+    ms = e0.elapsed_time(e1)
+    ms = max_over_ranks(world, ms)
+    ws.check("timed region")
+    time.sleep(0.3)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0 - 0.05, t_wall1 + 0.05)
+
+    # end to end: pinned host x -> device, block, device y -> pinned host
+    x_pin = torch.from_numpy(x_host.view(np.int16)).pin_memory()
+    y_pin = torch.empty(B, D_MODEL, dtype=torch.int16).pin_memory()
+    x_e = torch.empty_like(x)
+    y_e = torch.empty_like(y)
+    for _ in range(3):
+        x_e.copy_(x_pin, non_blocking=True)
+        uw.mlp_block(*dms, pipes, x_e, y_e, ws, stream)
+        y_pin.copy_(y_e, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.steps):
+        x_e.copy_(x_pin, non_blocking=True)
+        uw.mlp_block(*dms, pipes, x_e, y_e, ws, stream)
+        y_pin.copy_(y_e, non_blocking=True)
+    f1.record(stream)
+    f1.synchronize()
+    e2e_ms = max_over_ranks(world, f0.elapsed_time(f1))
+
+    # uncompressed BF16 comparator (cuBLAS through torch.matmul) on the same shapes
+    wt = [torch.from_numpy(w.view(np.int16)).to(dev).view(torch.bfloat16) for w in mats]
+    xb = x.view(torch.bfloat16)
+
+    def step_bf16():
+        g = xb @ wt[0].T
+        u = xb @ wt[1].T
+        h = torch.nn.functional.silu(g) * u
+        return h @ wt[2].T
+
+    for _ in range(3):
+        step_bf16()
+    torch.cuda.synchronize(dev)
+    g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g0.record(stream)
+    for _ in range(args.steps):
+        step_bf16()
+    g1.record(stream)
+    g1.synchronize()
+    bf16_ms = g0.elapsed_time(g1) / args.steps
+    del wt
+
+    # roofline of the dominant kernel (the reconstructive GEMM: every launch of
+    # the step is one)
+    peaks, src = measured_peaks()
+    per_step_bytes = sum(dm.direct_palette_bytes() for dm in dms) + 2 * B * (D_MODEL + FFN) * 2 + 2 * B * FFN * 2
+    t_step = ms / 1e3 / args.steps
+    achieved = per_step_bytes / t_step / 1e9
+    peak = float(peaks["hbm_gbs"])
+    weight_gbs = sum(2 * e.rows * e.cols for e in encs) / t_step / 1e9
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": B * args.steps * world / (ms / 1e3),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": dict(config_dict(args), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": NCU_TRAFFIC_PER_LAUNCH,
+                         "kernel": "gemm_kernel<IDX4 uniform palette> (3 launches per step)",
+                         "algorithmic_bytes_per_step": per_step_bytes, "peak_source": f"{src} hbm_gbs"},
+            "effective_weight_gbs": weight_gbs,
+            "bf16_torch_matmul_ms_per_step": bf16_ms,
+            "speedup_vs_bf16_torch": bf16_ms / (ms / args.steps),
+            "e2e": {"value": B * args.steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": B * D_MODEL * 2, "d2h_bytes_per_step": B * D_MODEL * 2},
+            "gpu_launches": int(launches),
+            "clocks": clocks,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                oracle_prepare(B, args.ref_fraction)
+                dt = min(oracle_block_sample(B, args.ref_fraction) for _ in range(3))
+            line["cpu_baseline"] = {
+                "value": B / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                "sample": f"best of 3 steps on {args.ref_fraction:.4f} of the rows of gate, up and down "
+                          f"(direct-palette rebuild + float64 GEMM), scaled to the full block; "
+                          f"os.cpu_count()={os.cpu_count()}"}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--batch", type=int, default=8)
+    ap.add_argument("--impl", default="uw", choices=["uw", "reference"])
+    ap.add_argument("--ref-fraction", type=float, default=1 / 16)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    world, rank, local = dist_init()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        return run_gpu(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

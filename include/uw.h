@@ -1,0 +1,327 @@
+/*
+ * uw.h -- C ABI of libuw: lossless Huffman-coded BF16 MLP weights and the
+ * reconstructive GEMM that consumes them, for NVIDIA B200 (sm_100a).
+ *
+ * The method is Cloudflare's "Unweight: how we compressed an LLM 22% without
+ * sacrificing quality":
+ *   - section "How to compress model weights effectively": a BF16 weight is
+ *     1 sign + 8 exponent + 7 mantissa bits; sign and mantissa stay raw; the
+ *     exponent is Huffman coded; the 16 most frequent exponents of a matrix
+ *     form its palette; a 64-element row holding any exponent outside the
+ *     palette is stored verbatim so the hot loop decides once per row;
+ *   - section "Four ways to use compressed weights": full decode, exponent-
+ *     only decode, run-time 4-bit palette transcode, and the same transcode
+ *     done at load time ("direct palette");
+ *   - section "Why no single pipeline wins": the best pipeline depends on the
+ *     matrix shape and the batch, so it is measured per matrix and batch;
+ *   - section "How the reconstructive matmul works": compressed tiles are
+ *     staged on chip, rebuilt to BF16 there and fed straight to the tensor
+ *     cores; decoded weights never go back to HBM.
+ *
+ * Storage layout of one compressed matrix W[rows, cols] (row-major, BF16,
+ * rows = output features, cols = input features, cols % 64 == 0):
+ *   group       64 consecutive elements of one row (the page's "64-element
+ *               row"); group g covers flat elements [64 g, 64 g + 64).
+ *   sm          uint8[rows*cols], one byte per element, dense (verbatim groups
+ *               included): byte k = (mantissa_k << 1) | sign_{k^1}; each byte
+ *               carries its own 7 mantissa bits and the sign of its pair
+ *               partner (elements 2j, 2j+1 of a row swap signs).  With this
+ *               layout two BF16 words are rebuilt from two sm bytes and two
+ *               exponent bytes by one byte permute and one 1-bit rotate.
+ *   stream      uint32[stream_words]: canonical Huffman codes of the palette
+ *               index of every element of every non-verbatim group, in group
+ *               order, packed MSB first (stream bit p = bit 31-(p%32) of word
+ *               p/32), followed by 2 zero words.
+ *   chunk_bit_off uint32[n_chunks+1]: a chunk is chunk_groups consecutive
+ *               groups; entry c is the stream bit where chunk c starts, the
+ *               last entry is the total bit count.  Chunks decode in parallel.
+ *   vflags      uint32[rows*words_per_row], words_per_row = ceil(cols/64/32):
+ *               bit (g%32) of word (row*words_per_row + g/32) is set when
+ *               group g of that row is verbatim.
+ *   vprefix     uint32[rows*words_per_row+1]: verbatim groups in all earlier
+ *               flag words (exclusive prefix); last entry = n_verbatim.
+ *   verbatim    uint16[n_verbatim*64]: the raw BF16 words of each verbatim
+ *               group, in group order.  The slot of group g of row r is
+ *               vprefix[w] + popcount(vflags[w] & ((1<<(g%32))-1)) with
+ *               w = r*words_per_row + g/32.
+ *   idx4        uint8[rows*cols/2] (optional, from uw_transcode_palette):
+ *               palette index per element, element 2j in the low nibble of
+ *               byte j of the row, 2j+1 in the high nibble; 0 in verbatim
+ *               groups.
+ *
+ * Conventions for every call:
+ *   - Every call returns a uw_status; nothing throws across the ABI.
+ *   - The caller owns all memory.  The library never allocates device
+ *     memory; device calls take a caller-provided workspace.
+ *   - Device calls are asynchronous on the given stream (a cudaStream_t
+ *     passed as void*, NULL = legacy default stream).  They return UW_OK once
+ *     launched.  Problems the GPU finds (a corrupt stream, a wait that ran
+ *     out of time) are recorded in the workspace's status word and read back
+ *     with uw_workspace_status().
+ *   - Host calls (uw_build_palette_codebook, uw_encode, uw_validate) are
+ *     synchronous and thread-safe.
+ *   - Device pointers must be 16-byte aligned; violations give
+ *     UW_ERR_INVALID_ARG before anything is launched.
+ */
+#ifndef UW_H
+#define UW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Exported symbols (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define UW_API __attribute__((visibility("default")))
+#else
+#define UW_API
+#endif
+
+typedef enum {
+  UW_OK = 0,
+  UW_ERR_INVALID_ARG = 1,        /* NULL/misaligned pointer, bad size or enum */
+  UW_ERR_UNSUPPORTED_SHAPE = 2,  /* cols % 64 != 0, batch out of range, ... */
+  UW_ERR_CORRUPT = 3,            /* stream or metadata inconsistent */
+  UW_ERR_TIMEOUT = 4,            /* a bounded on-GPU wait ran out */
+  UW_ERR_CUDA = 5,               /* a CUDA runtime call failed */
+  UW_ERR_WORKSPACE_TOO_SMALL = 6,
+  UW_ERR_NO_DEVICE = 7           /* no sm_100 device available */
+} uw_status;
+
+/* Execution pipelines (section "Four ways to use compressed weights").
+ * UW_PIPE_BF16 is the uncompressed comparator: the same GEMM kernel fed an
+ * already-BF16 matrix. */
+typedef enum {
+  UW_PIPE_FULL = 0,       /* Huffman -> BF16 in HBM, then GEMM on BF16 */
+  UW_PIPE_EXPONENT = 1,   /* Huffman -> exponent bytes, GEMM rebuilds from sm + exp8 */
+  UW_PIPE_TRANSCODE = 2,  /* Huffman -> 4-bit indices at run time, reconstructive GEMM */
+  UW_PIPE_DIRECT = 3,     /* 4-bit indices built at load time, reconstructive GEMM */
+  UW_PIPE_BF16 = 4        /* uncompressed BF16 matrix (comparator only) */
+} uw_pipeline;
+
+#define UW_GROUP 64
+#define UW_PALETTE 16
+#define UW_MAX_BATCH 512
+#define UW_MAX_CODE_LEN 15
+
+/* Palette and canonical Huffman code of one matrix. */
+typedef struct {
+  uint8_t palette[UW_PALETTE];   /* exponent value of each palette index */
+  uint8_t code_len[UW_PALETTE];  /* code length per index, 0 = no code */
+  uint16_t code[UW_PALETTE];     /* canonical code value (right aligned) */
+  uint64_t freq[UW_PALETTE];     /* count of each index over non-verbatim groups */
+  uint8_t n_symbols;             /* indices with a code */
+  uint8_t max_len;               /* longest code length (<= 15) */
+  uint8_t reserved[6];
+} uw_codebook;
+
+/* Sizes of every array of one compressed matrix. */
+typedef struct {
+  int64_t rows, cols;
+  int32_t chunk_groups;     /* groups per chunk (1..16) */
+  int32_t words_per_row;    /* vflags words per row */
+  int64_t n_groups;         /* rows*cols/64 */
+  int64_t n_chunks;         /* ceil(n_groups/chunk_groups) */
+  int64_t n_verbatim;       /* verbatim groups */
+  int64_t stream_words;     /* including the 2 trailing zero words */
+  int64_t total_bits;       /* coded bits (== chunk_bit_off[n_chunks]) */
+} uw_layout;
+
+/* One compressed matrix resident on the GPU: device pointers owned by the
+ * caller (layout and codebook by value).  idx4 may be NULL until
+ * uw_transcode_palette has filled a buffer for it. */
+typedef struct {
+  uw_layout L;
+  uw_codebook cb;
+  const uint8_t* sm;
+  const uint32_t* stream;
+  const uint32_t* chunk_bit_off;
+  const uint32_t* vflags;
+  const uint32_t* vprefix;
+  const uint16_t* verbatim;  /* may be NULL when n_verbatim == 0 */
+  const uint8_t* idx4;       /* may be NULL */
+} uw_matrix;
+
+/* ---------------------------------------------------------------------------
+ * Offline (host) calls
+ * ------------------------------------------------------------------------- */
+
+/* Palette + canonical Huffman code of a BF16 matrix (section "How to
+ * compress model weights effectively").  w_host: host uint16[rows*cols],
+ * row-major BF16 bits.  Palette = 16 most frequent exponents over the whole
+ * matrix, ties to the smaller value, free slots filled with unused values in
+ * ascending order.  Frequencies are counted over non-verbatim groups only;
+ * code lengths come from the two-smallest-merge construction with ties broken
+ * by (weight, node id), leaves 0..15, merged nodes 16, 17, ... in order.
+ * Errors: UW_ERR_INVALID_ARG (NULL), UW_ERR_UNSUPPORTED_SHAPE (cols % 64,
+ * rows < 1). */
+UW_API uw_status uw_build_palette_codebook(const uint16_t* w_host, int64_t rows, int64_t cols,
+                                    uw_codebook* out);
+
+/* Encode a matrix into the storage layout above (sections "How to compress
+ * model weights effectively" and "How the reconstructive matmul works").
+ * cb: from uw_build_palette_codebook (or any codebook whose codes cover
+ * every palette index used outside verbatim groups).  io_layout: filled on
+ * return.  When every output pointer is NULL the call only computes the sizes
+ * (io_layout) and returns; otherwise every output must be a host buffer of
+ * the size io_layout gives (verbatim may be NULL when n_verbatim == 0).
+ * Errors: UW_ERR_INVALID_ARG, UW_ERR_UNSUPPORTED_SHAPE (cols % 64, chunk_groups
+ * outside 1..16, more than 2^32-1 stream bits), UW_ERR_CORRUPT (codebook does
+ * not cover a used symbol). */
+UW_API uw_status uw_encode(const uint16_t* w_host, int64_t rows, int64_t cols, const uw_codebook* cb,
+                    int32_t chunk_groups, uw_layout* io_layout, uint8_t* sm, uint32_t* stream,
+                    uint32_t* chunk_bit_off, uint32_t* vflags, uint32_t* vprefix,
+                    uint16_t* verbatim);
+
+/* Host-side consistency check of a compressed matrix whose pointers are
+ * HOST copies: canonical codebook with Kraft sum <= 1, offsets monotone and
+ * ending at total_bits, vprefix equal to the running popcount of vflags,
+ * sizes consistent.  Run it before uploading data from an untrusted file.
+ * Errors: UW_ERR_INVALID_ARG, UW_ERR_CORRUPT. */
+UW_API uw_status uw_validate(const uw_matrix* host_mirror);
+
+/* ---------------------------------------------------------------------------
+ * Workspace
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of device workspace a device call needs for this matrix, pipeline
+ * and batch (batch 0 for the decode/transcode calls).  The workspace holds a
+ * status word, split-K partial sums and tile counters, and for the FULL /
+ * EXPONENT / TRANSCODE pipelines the intermediate decoded matrix.  Returns 0
+ * for invalid arguments. */
+UW_API size_t uw_workspace_bytes(const uw_layout* L, int32_t pipeline, int32_t batch);
+
+/* Zero a workspace (stream-ordered).  A workspace must be zeroed once before
+ * its first use; afterwards every call leaves its counters at zero again.
+ * Calls that share one workspace must be ordered on one stream. */
+UW_API uw_status uw_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronize the stream, read the workspace's sticky status word (the
+ * first problem any kernel recorded since the last read) and clear it. */
+UW_API uw_status uw_workspace_status(void* workspace, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Preprocessing kernels (section "Four ways to use compressed weights")
+ * ------------------------------------------------------------------------- */
+
+/* Full Huffman decode: out_bf16[rows*cols] (device, row-major BF16 bits)
+ * gets back every original word bit for bit, verbatim groups copied from the
+ * verbatim store.  Reads sm + stream + offsets + flags + verbatim; writes
+ * 2 bytes per element.  A chunk whose code lengths do not end exactly at
+ * the next chunk's offset records UW_ERR_CORRUPT. */
+UW_API uw_status uw_decode_full(const uw_matrix* m, uint16_t* out_bf16, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+/* Exponent-only decode: out_exp8[rows*cols] (device) = exponent byte of every
+ * element (verbatim groups from the verbatim store); half of the full
+ * decode's write traffic.  The GEMM recombines it with the raw sm bytes. */
+UW_API uw_status uw_decode_exponent_only(const uw_matrix* m, uint8_t* out_exp8, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/* Palette transcode: out_idx4[rows*cols/2] (device) = 4-bit palette index per
+ * element in the idx4 layout, 0 in verbatim groups; a quarter of the full
+ * decode's write traffic.  Run once at load time this is the "direct
+ * palette" preparation; run per call it is the "palette transcode"
+ * pipeline. */
+UW_API uw_status uw_transcode_palette(const uw_matrix* m, uint8_t* out_idx4, void* workspace,
+                               size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Reconstructive GEMM (section "How the reconstructive matmul works")
+ * ------------------------------------------------------------------------- */
+
+/* y = x W^T with the direct-palette matrix: x is device BF16 [batch, cols]
+ * row-major, y is device BF16 [batch, rows] row-major.  W is rebuilt tile by
+ * tile on chip from sm + idx4 (+ verbatim rows, chosen once per 64-element
+ * row) and fed to tcgen05 MMA with FP32 accumulation in tensor memory; y is
+ * rounded to nearest-even BF16.  m->idx4 must be set.  The split of the K
+ * loop across CTAs and the order of its reduction depend only on (rows, cols,
+ * batch, SM count), so all pipelines give bit-identical y.
+ * batch: 1..512.  Errors: UW_ERR_INVALID_ARG, UW_ERR_UNSUPPORTED_SHAPE,
+ * UW_ERR_WORKSPACE_TOO_SMALL, UW_ERR_CUDA. */
+UW_API uw_status uw_gemm_direct_palette(const uw_matrix* m, const uint16_t* x, int32_t batch,
+                                 uint16_t* y, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/* y = x W^T through any pipeline, including its preprocessing kernel (whose
+ * output lives in the workspace).  UW_PIPE_BF16 is not accepted here (see
+ * uw_gemm_bf16). */
+UW_API uw_status uw_gemm(const uw_matrix* m, int32_t pipeline, const uint16_t* x, int32_t batch,
+                  uint16_t* y, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Same as uw_gemm_direct_palette, but always uses the general palette lookup
+ * (the one for palettes whose used exponents differ in their top bit)
+ * instead of the faster single-table lookup.  Results are identical; this
+ * entry point exists so the general lookup can be tested on any matrix. */
+UW_API uw_status uw_gemm_direct_palette_general_lookup(const uw_matrix* m, const uint16_t* x,
+                                                       int32_t batch, uint16_t* y, void* workspace,
+                                                       size_t workspace_bytes, void* stream);
+
+/* Uncompressed comparator: y = x W^T with W given as device BF16
+ * [rows, cols]; the same GEMM kernel, loader reading BF16 tiles.  Workspace:
+ * uw_workspace_bytes with UW_PIPE_BF16. */
+UW_API uw_status uw_gemm_bf16(const uint16_t* w, int64_t rows, int64_t cols, const uint16_t* x,
+                       int32_t batch, uint16_t* y, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/* ---------------------------------------------------------------------------
+ * MLP block
+ * ------------------------------------------------------------------------- */
+
+/* h = bf16(SiLU(g) * u) elementwise over n BF16 values (device), computed in
+ * FP32: SiLU(v) = v / (1 + exp(-v)). */
+UW_API uw_status uw_swiglu(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t n, void* stream);
+
+/* One SwiGLU MLP block: y = W_down (SiLU(W_gate x) * (W_up x)).  gate, up:
+ * [ffn, d]; down: [d, ffn]; x: [batch, d]; y: [batch, d] (device BF16).
+ * pipelines[3]: pipeline per matrix (gate, up, down), e.g. from uw_autotune.
+ * The up GEMM applies SiLU(g)*u in its epilogue and writes h directly.
+ * Workspace: uw_mlp_workspace_bytes. */
+UW_API size_t uw_mlp_workspace_bytes(const uw_matrix* gate, const uw_matrix* up, const uw_matrix* down,
+                              const int32_t* pipelines, int32_t batch);
+UW_API uw_status uw_mlp_block(const uw_matrix* gate, const uw_matrix* up, const uw_matrix* down,
+                       const int32_t* pipelines, const uint16_t* x, int32_t batch, uint16_t* y,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Autotuner (sections "Key Points" and "Why no single pipeline wins")
+ * ------------------------------------------------------------------------- */
+
+/* Time every pipeline on this matrix at each batch and pick the fastest.
+ * For each batch b in batches[0..n_batches): warm up, then run reps timed
+ * calls (CUDA events on `stream`, preprocessing included), and keep the
+ * median.  out_us[i*4 + p] = median microseconds of pipeline p at batches[i]
+ * (+INF when the pipeline is unavailable, e.g. DIRECT without m->idx4);
+ * out_choice[i] = the pipeline with the smallest time.  x/y: device buffers
+ * of at least max(batches)*cols / max(batches)*rows BF16 values used as
+ * inputs/outputs of the timed calls.  flush/flush_bytes (optional, may be
+ * NULL/0): a device buffer larger than L2 that is overwritten before every
+ * timed call so the weights are read from HBM as they are in a real decode
+ * step.  Synchronizes `stream`.  Workspace: the maximum of
+ * uw_workspace_bytes over the four pipelines and batches. */
+UW_API uw_status uw_autotune(const uw_matrix* m, const int32_t* batches, int32_t n_batches,
+                      int32_t reps, const uint16_t* x, uint16_t* y, void* flush,
+                      size_t flush_bytes, void* workspace, size_t workspace_bytes,
+                      int32_t* out_choice, float* out_us, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Misc
+ * ------------------------------------------------------------------------- */
+
+UW_API const char* uw_status_string(uw_status s);
+
+/* Library version: major*10000 + minor*100 + patch. */
+UW_API int32_t uw_version(void);
+
+/* Number of kernel launches the library has issued in this process (all
+ * devices); used to count launches inside a timed region. */
+UW_API uint64_t uw_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* UW_H */

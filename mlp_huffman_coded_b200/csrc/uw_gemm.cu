@@ -1,0 +1,863 @@
+// Reconstructive GEMM on tcgen05 tensor cores, the SwiGLU glue and the MLP
+// block.
+//
+// Method: Cloudflare, "Unweight: how we compressed an LLM 22% without
+// sacrificing quality", section "How the reconstructive matmul works":
+// compressed tiles (sign+mantissa bytes, exponent data or palette indices,
+// and the verbatim rows of rare-exponent 64-element rows) are staged into
+// shared memory by TMA running ahead in a ring; other threads rebuild BF16 on
+// chip and feed it straight to the tensor cores, so decoded weights never go
+// back to HBM.  Section "Four ways to use compressed weights" gives the four
+// pipelines; they differ only in the tile loader of this one kernel.
+//
+// Blackwell design (what differs from the page's Hopper TMA/WGMMA kernel):
+//  * W is the MMA's A operand (M = 128 output rows per tile), the token batch
+//    is the N side (16..256 columns), so a decode-time batch of 1..16 is one
+//    N = 16 MMA.
+//  * Rebuilt BF16 goes from registers into tensor memory (tcgen05.st) and the
+//    MMA reads A from TMEM; shared memory only carries the compressed tiles
+//    and the activation tile.  This keeps shared-memory traffic near 2.3
+//    bytes per weight instead of ~7 with an SMEM round trip.
+//  * One rebuild thread owns one weight row (= one TMEM lane) per k-block of
+//    64 elements, i.e. exactly one 64-element group, so the verbatim check is
+//    one flag bit per row per k-block and never per element.
+//  * Persistent CTAs, one per SM, split the linearised (tile, k-block) space
+//    evenly (stream-K); a tile split across CTAs is reduced in CTA order by
+//    the last CTA to finish it, so the result does not depend on timing and
+//    is identical for every pipeline.
+//  * FP32 accumulators live in TMEM; the epilogue reads them with tcgen05.ld
+//    and rounds to nearest-even BF16 (optionally applying SiLU(g) * u).
+//  * Every barrier wait is bounded in time; a timeout records UW_ERR_TIMEOUT,
+//    drains in-flight copies and frees tensor memory before returning.
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "uw_device.cuh"
+#include "uw_internal.h"
+
+namespace uw {
+
+namespace {
+
+constexpr int kThreads = 320;  // 10 warps
+constexpr int kWarpProducer = 0;
+constexpr int kWarpMma = 1;
+constexpr int kWarpRebuild0 = 2;  // warps 2..5
+constexpr int kWarpEpi0 = 6;      // warps 6..9
+constexpr int kVCap = 16;         // verbatim rows staged on chip per tile
+constexpr int kMaxStages = 8;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCol = 0;
+constexpr uint32_t kAStageCol0 = 256;
+constexpr size_t kSmemLimit = 227 * 1024;
+constexpr size_t kSmemFloor = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
+
+enum KernelLoader { kBF16 = 0, kEXP8 = 1, kIDX4U = 2, kIDX4M = 3 };
+
+struct KParams {
+  int N, K, B, KB, n_ntiles, ntile;
+  long long units;
+  int grid;
+  int stages;
+  uint32_t stage_bytes, off_x, off_wa, off_wb, off_verb, off_hdr;
+  uint32_t x_bytes, wa_bytes, wb_bytes;
+  uint32_t meta_off, meta_slot_words;  // per slot: flags then prefixes
+  uint32_t bar_off;
+  int wpr;
+  const uint32_t* vflags;
+  const uint32_t* vprefix;
+  const uint16_t* verbatim;
+  uint16_t* y;
+  const uint16_t* gate;
+  float* partials;
+  uint32_t* counters;
+  uint32_t* status;
+  PaletteTables pal;
+  uint32_t idesc;
+};
+
+struct Bars {
+  uint64_t full[kMaxStages];
+  uint64_t rebuilt[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t acc_full, acc_empty, drain;
+  uint64_t meta_full[2];
+  uint32_t tmem_base;
+  uint32_t abort;
+  uint32_t is_last;
+};
+
+__device__ __forceinline__ int64_t unit_begin(int64_t c, const KParams& p) {
+  return c * p.units / p.grid;
+}
+// CTA whose unit range holds unit u
+__device__ __forceinline__ int64_t unit_owner(int64_t u, const KParams& p) {
+  return ((u + 1) * p.grid - 1) / p.units;
+}
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* b, uint32_t* status) {
+  const bool ok = mbar_wait(bar, parity, &b->abort, status);
+  return __all_sync(0xFFFFFFFFu, ok);
+}
+
+__device__ __forceinline__ bool group_and(bool v) {  // warps 6..9 (named barrier 1)
+  uint32_t out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(out)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return out != 0;
+}
+__device__ __forceinline__ void group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+
+// ----------------------------- tile rebuild ---------------------------------
+// Each rebuild thread owns one row r of the 128-row tile and produces the 64
+// BF16 values of the current k-block as 32 packed words (element 2i in the
+// low half of word i), ready for tcgen05.st.  Tile rows come from TMA with a
+// swizzle that keeps these row-per-thread 16-byte reads bank-conflict free.
+
+template <int L>
+__device__ __forceinline__ void rebuild_row(const uint8_t* stage, const KParams& p, int r, uint32_t (&o)[32]) {
+  if constexpr (L == kBF16) {
+    const uint8_t* t = stage + p.off_wa;  // rows of 128 B, 128-byte swizzle
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint4 v = lds128(t + r * 128 + ((j ^ (r & 7)) << 4));
+      o[4 * j] = v.x;
+      o[4 * j + 1] = v.y;
+      o[4 * j + 2] = v.z;
+      o[4 * j + 3] = v.w;
+    }
+  } else if constexpr (L == kEXP8) {
+    const uint8_t* ts = stage + p.off_wa;  // sm rows of 64 B, 64-byte swizzle
+    const uint8_t* te = stage + p.off_wb;  // exponent rows of 64 B, 64-byte swizzle
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = (j ^ ((r >> 1) & 3)) << 4;
+      const uint4 s = lds128(ts + r * 64 + c);
+      const uint4 e = lds128(te + r * 64 + c);
+      rebuild4(s.x, e.x, o[8 * j + 0], o[8 * j + 1]);
+      rebuild4(s.y, e.y, o[8 * j + 2], o[8 * j + 3]);
+      rebuild4(s.z, e.z, o[8 * j + 4], o[8 * j + 5]);
+      rebuild4(s.w, e.w, o[8 * j + 6], o[8 * j + 7]);
+    }
+  } else {
+    const uint8_t* ts = stage + p.off_wa;  // sm rows of 64 B, 64-byte swizzle
+    const uint8_t* ti = stage + p.off_wb;  // index rows of 32 B, 32-byte swizzle
+    uint32_t iw[8];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const uint4 v = lds128(ti + r * 32 + ((j ^ ((r >> 2) & 1)) << 4));
+      iw[4 * j] = v.x;
+      iw[4 * j + 1] = v.y;
+      iw[4 * j + 2] = v.z;
+      iw[4 * j + 3] = v.w;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 s = lds128(ts + r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+      const uint32_t sw[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const uint32_t nib = iw[2 * j + h];  // 8 indices: elements 16j + 8h .. +7
+        uint32_t e0, e1;
+        if constexpr (L == kIDX4U) {
+          e0 = lookup4_uniform(p.pal, nib);
+          e1 = lookup4_uniform(p.pal, nib >> 16);
+        } else {
+          e0 = lookup4_mixed(p.pal, nib);
+          e1 = lookup4_mixed(p.pal, nib >> 16);
+        }
+        rebuild4(sw[2 * h], e0, o[8 * j + 4 * h + 0], o[8 * j + 4 * h + 1]);
+        rebuild4(sw[2 * h + 1], e1, o[8 * j + 4 * h + 2], o[8 * j + 4 * h + 3]);
+      }
+    }
+  }
+}
+
+// ------------------------------- the kernel ----------------------------------
+template <int L>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wa,
+                const __grid_constant__ CUtensorMap tm_wb, const KParams p) {
+  constexpr bool kIdx4 = (L == kIDX4U || L == kIDX4M);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Bars* bars = reinterpret_cast<Bars*>(smem + p.bar_off);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t u0 = unit_begin(blockIdx.x, p);
+  const int64_t u1 = unit_begin(blockIdx.x + 1, p);
+  const int S = p.stages;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->rebuilt[s], 4);
+      mbar_init(&bars->empty[s], 1);
+    }
+    mbar_init(&bars->acc_full, 1);
+    mbar_init(&bars->acc_empty, 4);
+    mbar_init(&bars->drain, 1);
+    mbar_init(&bars->meta_full[0], 1);
+    mbar_init(&bars->meta_full[1], 1);
+    bars->abort = 0;
+    bars->is_last = 0;
+    mbar_fence_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(&bars->tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kWarpProducer && lane == 0) {
+    prefetch_tensormap(&tm_x);
+    prefetch_tensormap(&tm_wa);
+    if (L != kBF16) prefetch_tensormap(&tm_wb);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == kWarpProducer) {
+    // ------------------------------ producer --------------------------------
+    const int mt_first = static_cast<int>((u0 / p.KB) / p.n_ntiles);
+    const int mt_last = static_cast<int>(((u1 - 1) / p.KB) / p.n_ntiles);
+    uint32_t* meta = reinterpret_cast<uint32_t*>(smem + p.meta_off);
+    int meta_issued[2] = {0, 0};
+    // per-m-tile verbatim flags and prefix counts for its 128 rows
+    auto issue_meta = [&](int mt, int slot) {
+      uint32_t* dst = meta + slot * 2 * p.meta_slot_words;
+      const int64_t row0 = static_cast<int64_t>(mt) * 128;
+      const int rows = static_cast<int>(p.N - row0 < 128 ? p.N - row0 : 128);
+      const uint32_t words = static_cast<uint32_t>(rows) * p.wpr;
+      const uint32_t bulk_words = words & ~3u;  // 16-byte multiple
+      if (lane == 0) {
+        const uint32_t tx = bulk_words ? 2 * bulk_words * 4 : 0;
+        mbar_arrive_expect_tx(&bars->meta_full[slot], tx);
+        if (bulk_words) {
+          bulk_load(dst, p.vflags + row0 * p.wpr, bulk_words * 4, &bars->meta_full[slot]);
+          bulk_load(dst + p.meta_slot_words, p.vprefix + row0 * p.wpr, bulk_words * 4, &bars->meta_full[slot]);
+        }
+      }
+      // tail words and rows past the matrix: plain loads / zeros
+      for (uint32_t w = bulk_words + lane; w < p.meta_slot_words; w += 32) {
+        dst[w] = w < words ? p.vflags[row0 * p.wpr + w] : 0u;
+        dst[p.meta_slot_words + w] = w < words ? p.vprefix[row0 * p.wpr + w] : 0u;
+      }
+      __syncwarp();
+      ++meta_issued[slot];
+    };
+    if (kIdx4) {
+      issue_meta(mt_first, 0);
+      if (mt_first + 1 <= mt_last) issue_meta(mt_first + 1, 1);
+    }
+    int cur_mt = -1;
+    int64_t i = 0;
+    for (int64_t u = u0; u < u1; ++u, ++i) {
+      const int s = static_cast<int>(i % S);
+      const uint32_t k = static_cast<uint32_t>(i / S);
+      if (k > 0 && !warp_wait(&bars->empty[s], (k - 1) & 1, bars, p.status)) break;
+      const int64_t t = u / p.KB;
+      const int kb = static_cast<int>(u - t * p.KB);
+      const int mt = static_cast<int>(t / p.n_ntiles);
+      const int nt = static_cast<int>(t - static_cast<int64_t>(mt) * p.n_ntiles);
+      uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
+      uint32_t tx = p.x_bytes + p.wa_bytes + p.wb_bytes;
+      int vq_dst[4];
+      int64_t vq_src[4];
+      if (kIdx4) {
+        const int j = mt - mt_first;
+        if (mt != cur_mt) {
+          if (j >= 1 && mt + 1 <= mt_last) issue_meta(mt + 1, (j + 1) & 1);
+          if (!warp_wait(&bars->meta_full[j & 1], (j >> 1) & 1, bars, p.status)) break;
+          cur_mt = mt;
+        }
+        const uint32_t* mf = meta + (j & 1) * 2 * p.meta_slot_words;
+        const uint32_t* mp = mf + p.meta_slot_words;
+        const int fwi = kb >> 5;
+        const uint32_t fbit = 1u << (kb & 31);
+        uint32_t* hdr = reinterpret_cast<uint32_t*>(stage + p.off_hdr);
+        int total = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int r = q * 32 + lane;
+          const uint32_t w = mf[r * p.wpr + fwi];
+          const bool v = (w & fbit) != 0;
+          const uint32_t m = __ballot_sync(0xFFFFFFFFu, v);
+          const int idx = total + __popc(m & ((1u << lane) - 1));
+          vq_dst[q] = (v && idx < kVCap) ? idx : -1;
+          vq_src[q] = static_cast<int64_t>(mp[r * p.wpr + fwi]) + __popc(w & (fbit - 1));
+          if (lane == 0) hdr[q] = m;
+          total += __popc(m);
+        }
+        tx += static_cast<uint32_t>(min(total, kVCap)) * 128u;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&bars->full[s], tx);
+        tma_load_2d(stage + p.off_x, &tm_x, kb * 64, nt * p.ntile, &bars->full[s]);
+        if (L == kIDX4U || L == kIDX4M) {
+          tma_load_2d(stage + p.off_wa, &tm_wa, kb * 64, mt * 128, &bars->full[s]);
+          tma_load_2d(stage + p.off_wb, &tm_wb, kb * 32, mt * 128, &bars->full[s]);
+        } else if (L == kEXP8) {
+          tma_load_2d(stage + p.off_wa, &tm_wa, kb * 64, mt * 128, &bars->full[s]);
+          tma_load_2d(stage + p.off_wb, &tm_wb, kb * 64, mt * 128, &bars->full[s]);
+        } else {
+          tma_load_2d(stage + p.off_wa, &tm_wa, kb * 64, mt * 128, &bars->full[s]);
+        }
+      }
+      __syncwarp();
+      if (kIdx4) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (vq_dst[q] >= 0)
+            bulk_load(stage + p.off_verb + vq_dst[q] * 128, p.verbatim + vq_src[q] * 64, 128, &bars->full[s]);
+      }
+    }
+    // drain: the last use of every stage and every issued flag load must land
+    // before the CTA can exit (normally already complete)
+    if (lane == 0) {
+      const int64_t issued = i;
+      for (int64_t q = issued - S > 0 ? issued - S : 0; q < issued; ++q)
+        mbar_wait(&bars->full[q % S], static_cast<uint32_t>(q / S) & 1, nullptr, p.status);
+      for (int sl = 0; sl < 2; ++sl)
+        if (meta_issued[sl] > 0) mbar_wait(&bars->meta_full[sl], (meta_issued[sl] - 1) & 1, nullptr, p.status);
+    }
+  } else if (warp == kWarpMma) {
+    // ----------------------------- MMA issuer -------------------------------
+    if (lane == 0) {
+      uint32_t seg = 0;
+      int64_t i = 0;
+      for (int64_t u = u0; u < u1; ++u, ++i) {
+        const int s = static_cast<int>(i % S);
+        const uint32_t k = static_cast<uint32_t>(i / S);
+        const int kb = static_cast<int>(u % p.KB);
+        const bool first = (u == u0) || kb == 0;
+        const bool last = (u == u1 - 1) || kb == p.KB - 1;
+        if (first && seg > 0) {
+          if (!mbar_wait(&bars->acc_empty, (seg - 1) & 1, &bars->abort, p.status)) break;
+          tc_fence_after();
+        }
+        if (!mbar_wait(&bars->full[s], k & 1, &bars->abort, p.status)) break;
+        if (!mbar_wait(&bars->rebuilt[s], k & 1, &bars->abort, p.status)) break;
+        tc_fence_after();
+        const uint32_t a_tmem = tmem + kAStageCol0 + static_cast<uint32_t>(s) * 32;
+        const uint64_t b_desc = smem_desc_sw128(smem_u32(smem + static_cast<size_t>(s) * p.stage_bytes + p.off_x));
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          mma_ts(tmem + kAccCol, a_tmem + j * 8, b_desc + static_cast<uint64_t>(j * 2), p.idesc,
+                 (first && j == 0) ? 0u : 1u);
+        tc_commit(&bars->empty[s]);
+        if (last) {
+          tc_commit(&bars->acc_full);
+          ++seg;
+        }
+      }
+      // every MMA issued so far must finish before tensor memory is freed
+      tc_commit(&bars->drain);
+      mbar_wait(&bars->drain, 0, nullptr, p.status);
+    }
+    __syncwarp();
+  } else if (warp < kWarpEpi0) {
+    // ------------------------------- rebuild --------------------------------
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    int64_t i = 0;
+    for (int64_t u = u0; u < u1; ++u, ++i) {
+      const int s = static_cast<int>(i % S);
+      const uint32_t k = static_cast<uint32_t>(i / S);
+      if (!warp_wait(&bars->full[s], k & 1, bars, p.status)) break;
+      tc_fence_after();
+      const uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
+      uint32_t o[32];
+      rebuild_row<L>(stage, p, r, o);
+      if (kIdx4) {
+        // verbatim rows: one flag bit per row and k-block, no per-element test
+        const uint32_t* hdr = reinterpret_cast<const uint32_t*>(stage + p.off_hdr);
+        const uint32_t m = hdr[q];
+        if ((m >> lane) & 1) {
+          int idx = __popc(m & ((1u << lane) - 1));
+          for (int qq = 0; qq < q; ++qq) idx += __popc(hdr[qq]);
+          const uint4* src;
+          if (idx < kVCap) {
+            src = reinterpret_cast<const uint4*>(stage + p.off_verb + idx * 128);
+          } else {
+            // more verbatim rows than staged slots: read this one from HBM
+            const int64_t t = u / p.KB;
+            const int kb = static_cast<int>(u - t * p.KB);
+            const int64_t n = (t / p.n_ntiles) * 128 + r;
+            const int64_t fw = n * p.wpr + (kb >> 5);
+            const uint32_t fl = p.vflags[fw];
+            const int64_t slot = static_cast<int64_t>(p.vprefix[fw]) + __popc(fl & ((1u << (kb & 31)) - 1));
+            src = reinterpret_cast<const uint4*>(p.verbatim + slot * 64);
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint4 v = src[j];
+            o[4 * j] = v.x;
+            o[4 * j + 1] = v.y;
+            o[4 * j + 2] = v.z;
+            o[4 * j + 3] = v.w;
+          }
+        }
+      }
+      tmem_st32(tmem + (static_cast<uint32_t>(q * 32) << 16) + kAStageCol0 + static_cast<uint32_t>(s) * 32, o);
+      tc_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->rebuilt[s]);
+    }
+  } else {
+    // ------------------------------- epilogue -------------------------------
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    uint32_t seg = 0;
+    int64_t u = u0;
+    while (u < u1) {
+      const int64_t t = u / p.KB;
+      const int64_t seg_end = u1 < (t + 1) * p.KB ? u1 : (t + 1) * p.KB;
+      const int mt = static_cast<int>(t / p.n_ntiles);
+      const int nt = static_cast<int>(t - static_cast<int64_t>(mt) * p.n_ntiles);
+      const int64_t c_first = unit_owner(t * p.KB, p);
+      const int64_t c_last = unit_owner(t * p.KB + p.KB - 1, p);
+      const int ncontrib = static_cast<int>(c_last - c_first + 1);
+      bool ok = mbar_wait(&bars->acc_full, seg & 1, &bars->abort, p.status);
+      ok = __all_sync(0xFFFFFFFFu, ok);
+      ok = group_and(ok);
+      if (!ok) break;
+      tc_fence_after();
+      const int64_t n = static_cast<int64_t>(mt) * 128 + r;
+      const bool row_ok = n < p.N;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + kAccCol;
+      const int64_t slot0 = t + c_first;
+      for (int cc = 0; cc < p.ntile / 16; ++cc) {
+        uint32_t v[16];
+        tmem_ld16(taddr + cc * 16, v);
+        tc_wait_ld();
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          const int col = cc * 16 + jj;
+          const int b = nt * p.ntile + col;
+          if (ncontrib == 1) {
+            if (row_ok && b < p.B) {
+              __nv_bfloat16 val = __float2bfloat16_rn(__uint_as_float(v[jj]));
+              if (p.gate) val = swiglu_bf16(reinterpret_cast<const __nv_bfloat16*>(p.gate)[static_cast<int64_t>(b) * p.N + n], val);
+              reinterpret_cast<__nv_bfloat16*>(p.y)[static_cast<int64_t>(b) * p.N + n] = val;
+            }
+          } else {
+            const int64_t slot = slot0 + (blockIdx.x - c_first);
+            p.partials[(slot * p.ntile + col) * 128 + r] = __uint_as_float(v[jj]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->acc_empty);
+      if (ncontrib > 1) {
+        __threadfence();
+        group_sync();
+        if (warp == kWarpEpi0 && lane == 0) {
+          const uint32_t old = atomicAdd(p.counters + t, 1u);
+          bars->is_last = (old == static_cast<uint32_t>(ncontrib - 1)) ? 1u : 0u;
+        }
+        group_sync();
+        if (bars->is_last) {
+          __threadfence();
+          for (int col = 0; col < p.ntile; ++col) {
+            const int b = nt * p.ntile + col;
+            if (!row_ok || b >= p.B) continue;
+            float acc = 0.0f;
+            for (int jc = 0; jc < ncontrib; ++jc) acc += __ldcg(p.partials + ((slot0 + jc) * p.ntile + col) * 128 + r);
+            __nv_bfloat16 val = __float2bfloat16_rn(acc);
+            if (p.gate) val = swiglu_bf16(reinterpret_cast<const __nv_bfloat16*>(p.gate)[static_cast<int64_t>(b) * p.N + n], val);
+            reinterpret_cast<__nv_bfloat16*>(p.y)[static_cast<int64_t>(b) * p.N + n] = val;
+          }
+          if (warp == kWarpEpi0 && lane == 0) p.counters[t] = 0;
+        }
+      }
+      ++seg;
+      u = seg_end;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+__global__ void swiglu_kernel(const __nv_bfloat16* __restrict__ g, const __nv_bfloat16* __restrict__ u,
+                              __nv_bfloat16* __restrict__ h, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    h[i] = swiglu_bf16(g[i], u[i]);
+}
+
+// ------------------------------ host side ------------------------------------
+
+struct Layout {
+  int stages = 0;
+  uint32_t stage_bytes = 0, off_x = 0, off_wa = 0, off_wb = 0, off_verb = 0, off_hdr = 0;
+  uint32_t x_bytes = 0, wa_bytes = 0, wb_bytes = 0;
+  uint32_t meta_off = 0, meta_slot_words = 0, bar_off = 0;
+  size_t smem = 0;
+};
+
+uint32_t a1024(uint32_t v) { return (v + 1023u) & ~1023u; }
+
+bool make_layout(int loader, int ntile, int wpr, Layout* out) {
+  Layout l;
+  l.x_bytes = static_cast<uint32_t>(ntile) * 128;
+  const bool idx4 = loader == kIDX4U || loader == kIDX4M;
+  l.wa_bytes = loader == kBF16 ? 16384u : 8192u;
+  l.wb_bytes = loader == kBF16 ? 0u : (loader == kEXP8 ? 8192u : 4096u);
+  l.off_x = 0;
+  l.off_wa = a1024(l.off_x + l.x_bytes);
+  l.off_wb = a1024(l.off_wa + l.wa_bytes);
+  l.off_verb = a1024(l.off_wb + l.wb_bytes);
+  l.off_hdr = l.off_verb + (idx4 ? kVCap * 128u : 0u);
+  l.stage_bytes = a1024(l.off_hdr + (idx4 ? 64u : 0u));
+  l.meta_slot_words = idx4 ? 128u * static_cast<uint32_t>(wpr) : 0u;
+  const uint32_t meta_bytes = a1024(2u * 2u * l.meta_slot_words * 4u);
+  const uint32_t fixed = meta_bytes + a1024(sizeof(Bars)) + 1024u;  // + alignment slack
+  int stages = static_cast<int>((kSmemLimit - fixed) / l.stage_bytes);
+  stages = std::min(stages, kMaxStages);
+  if (stages < 2) return false;
+  l.stages = stages;
+  l.meta_off = static_cast<uint32_t>(stages) * l.stage_bytes;
+  l.bar_off = l.meta_off + meta_bytes;
+  l.smem = std::max<size_t>(static_cast<size_t>(l.bar_off) + a1024(sizeof(Bars)) + 1024u, kSmemFloor);
+  *out = l;
+  return true;
+}
+
+template <int L>
+uw_status launch_kernel(const CUtensorMap& x, const CUtensorMap& wa, const CUtensorMap& wb, const KParams& kp,
+                        size_t smem, cudaStream_t s) {
+  static std::once_flag once[64];
+  static cudaError_t attr_err[64];
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::call_once(once[dev & 63], [&] {
+    attr_err[dev & 63] = cudaFuncSetAttribute(gemm_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              static_cast<int>(kSmemLimit));
+  });
+  if (attr_err[dev & 63] != cudaSuccess) return UW_ERR_CUDA;
+  gemm_kernel<L><<<kp.grid, kThreads, smem, s>>>(x, wa, wb, kp);
+  note_launch();
+  return cuda_status(cudaGetLastError());
+}
+
+PaletteTables palette_tables(const uint8_t* pal, const uint8_t* code_len, bool* mixed) {
+  PaletteTables t;
+  uint32_t w[4] = {0, 0, 0, 0}, b7[4] = {0, 0, 0, 0};
+  int seen0 = 0, seen1 = 0;
+  for (int i = 0; i < 16; ++i) {
+    w[i / 4] |= static_cast<uint32_t>(pal[i] | 0x80u) << (8 * (i % 4));
+    b7[i / 4] |= static_cast<uint32_t>(0xBFu | ((pal[i] >> 7) << 6)) << (8 * (i % 4));
+    if (!code_len || code_len[i]) {
+      if (pal[i] & 0x80) seen1 = 1;
+      else seen0 = 1;
+    }
+  }
+  t.lo0 = w[0];
+  t.lo1 = w[1];
+  t.hi0 = w[2];
+  t.hi1 = w[3];
+  t.b7lo0 = b7[0];
+  t.b7lo1 = b7[1];
+  t.b7hi0 = b7[2];
+  t.b7hi1 = b7[3];
+  *mixed = seen0 && seen1;
+  t.keep = seen1 ? 0xFFFFFFFFu : 0x7F7F7F7Fu;
+  return t;
+}
+
+}  // namespace
+
+uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
+  DeviceInfo dev;
+  uw_status st = device_info(&dev);
+  if (st != UW_OK) return st;
+  GemmPlan plan;
+  if ((st = gemm_plan(a.N, a.K, a.B, dev.sm_count, &plan)) != UW_OK) return st;
+  if (!a.x || !a.y || !a.ws || !aligned16(a.x) || !aligned16(a.ws)) return UW_ERR_INVALID_ARG;
+  if (a.ws_bytes < gemm_ws_bytes(plan)) return UW_ERR_WORKSPACE_TOO_SMALL;
+  int kl;
+  PaletteTables pal{};
+  if (a.loader == kLoaderBF16) {
+    if (!a.wbf16 || !aligned16(a.wbf16)) return UW_ERR_INVALID_ARG;
+    kl = kBF16;
+  } else if (a.loader == kLoaderEXP8) {
+    if (!a.sm || !a.aux || !aligned16(a.sm) || !aligned16(a.aux)) return UW_ERR_INVALID_ARG;
+    kl = kEXP8;
+  } else {
+    if (!a.sm || !a.aux || !a.vflags || !a.vprefix || !a.palette) return UW_ERR_INVALID_ARG;
+    if (!aligned16(a.sm) || !aligned16(a.aux) || !aligned16(a.vflags) || !aligned16(a.vprefix) ||
+        (a.verbatim && !aligned16(a.verbatim)))
+      return UW_ERR_INVALID_ARG;
+    bool mixed = false;
+    pal = palette_tables(a.palette, a.code_len, &mixed);
+    kl = (mixed || a.force_mixed_palette) ? kIDX4M : kIDX4U;
+  }
+  Layout lay;
+  if (!make_layout(kl, plan.ntile, a.wpr, &lay)) return UW_ERR_UNSUPPORTED_SHAPE;
+
+  CUtensorMap tx, twa, twb;
+  std::memset(&twb, 0, sizeof(twb));
+  if ((st = make_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, a.K, a.B, a.K * 2, 64, plan.ntile,
+                               CU_TENSOR_MAP_SWIZZLE_128B)) != UW_OK)
+    return st;
+  if (kl == kBF16) {
+    if ((st = make_tensor_map_2d(&twa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.wbf16, a.K, a.N, a.K * 2, 64, 128,
+                                 CU_TENSOR_MAP_SWIZZLE_128B)) != UW_OK)
+      return st;
+    twb = twa;
+  } else {
+    if ((st = make_tensor_map_2d(&twa, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.sm, a.K, a.N, a.K, 64, 128,
+                                 CU_TENSOR_MAP_SWIZZLE_64B)) != UW_OK)
+      return st;
+    if (kl == kEXP8)
+      st = make_tensor_map_2d(&twb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.aux, a.K, a.N, a.K, 64, 128,
+                              CU_TENSOR_MAP_SWIZZLE_64B);
+    else
+      st = make_tensor_map_2d(&twb, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.aux, a.K / 2, a.N, a.K / 2, 32, 128,
+                              CU_TENSOR_MAP_SWIZZLE_32B);
+    if (st != UW_OK) return st;
+  }
+
+  KParams kp;
+  std::memset(&kp, 0, sizeof(kp));
+  kp.N = static_cast<int>(a.N);
+  kp.K = static_cast<int>(a.K);
+  kp.B = a.B;
+  kp.KB = plan.KB;
+  kp.n_ntiles = plan.n_ntiles;
+  kp.ntile = plan.ntile;
+  kp.units = plan.units;
+  kp.grid = plan.grid;
+  kp.stages = lay.stages;
+  kp.stage_bytes = lay.stage_bytes;
+  kp.off_x = lay.off_x;
+  kp.off_wa = lay.off_wa;
+  kp.off_wb = lay.off_wb;
+  kp.off_verb = lay.off_verb;
+  kp.off_hdr = lay.off_hdr;
+  kp.x_bytes = lay.x_bytes;
+  kp.wa_bytes = lay.wa_bytes;
+  kp.wb_bytes = lay.wb_bytes;
+  kp.meta_off = lay.meta_off;
+  kp.meta_slot_words = lay.meta_slot_words;
+  kp.bar_off = lay.bar_off;
+  kp.wpr = a.wpr;
+  kp.vflags = a.vflags;
+  kp.vprefix = a.vprefix;
+  kp.verbatim = a.verbatim;
+  kp.y = a.y;
+  kp.gate = a.gate;
+  uint8_t* ws = static_cast<uint8_t*>(a.ws);
+  kp.status = reinterpret_cast<uint32_t*>(ws);
+  kp.counters = reinterpret_cast<uint32_t*>(ws + kWsHeader);
+  kp.partials = reinterpret_cast<float*>(ws + kWsHeader + plan.counter_bytes);
+  kp.pal = pal;
+  kp.idesc = idesc_bf16_f32(plan.ntile);
+
+  switch (kl) {
+    case kBF16: return launch_kernel<kBF16>(tx, twa, twb, kp, lay.smem, s);
+    case kEXP8: return launch_kernel<kEXP8>(tx, twa, twb, kp, lay.smem, s);
+    case kIDX4U: return launch_kernel<kIDX4U>(tx, twa, twb, kp, lay.smem, s);
+    default: return launch_kernel<kIDX4M>(tx, twa, twb, kp, lay.smem, s);
+  }
+}
+
+uw_status launch_swiglu(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t n, cudaStream_t s) {
+  if (n < 0 || (n > 0 && (!g || !u || !h))) return UW_ERR_INVALID_ARG;
+  if (n == 0) return UW_OK;
+  DeviceInfo dev;
+  uw_status st = device_info(&dev);
+  if (st != UW_OK) return st;
+  const int64_t blocks = std::min<int64_t>((n + 255) / 256, static_cast<int64_t>(dev.sm_count) * 16);
+  swiglu_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(reinterpret_cast<const __nv_bfloat16*>(g),
+                                                          reinterpret_cast<const __nv_bfloat16*>(u),
+                                                          reinterpret_cast<__nv_bfloat16*>(h), n);
+  note_launch();
+  return cuda_status(cudaGetLastError());
+}
+
+}  // namespace uw
+
+using namespace uw;
+
+namespace {
+
+// Runs one GEMM of matrix m through `pipeline`.  ws: header + counters +
+// partials; scratch: the pipeline's intermediate matrix (may alias nothing
+// else that is live).
+uw_status run_pipeline(const uw_matrix* m, int pipeline, const uint16_t* x, int32_t batch, uint16_t* y,
+                       const uint16_t* gate, void* ws, size_t ws_bytes, void* scratch, size_t scratch_bytes,
+                       cudaStream_t s, int force_mixed = 0) {
+  uw_status st = check_matrix(m);
+  if (st != UW_OK) return st;
+  if (pipeline < UW_PIPE_FULL || pipeline > UW_PIPE_DIRECT) return UW_ERR_INVALID_ARG;
+  GemmArgs a;
+  a.N = m->L.rows;
+  a.K = m->L.cols;
+  a.B = batch;
+  a.x = x;
+  a.y = y;
+  a.gate = gate;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  a.wpr = m->L.words_per_row;
+  a.force_mixed_palette = force_mixed;
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  const size_t need = pipeline_scratch_bytes(&m->L, pipeline);
+  if (pipeline != UW_PIPE_DIRECT && (!scratch || scratch_bytes < need)) return UW_ERR_WORKSPACE_TOO_SMALL;
+  switch (pipeline) {
+    case UW_PIPE_FULL:
+      if ((st = launch_decode(m, 0, scratch, status, s)) != UW_OK) return st;
+      a.loader = kLoaderBF16;
+      a.wbf16 = static_cast<const uint16_t*>(scratch);
+      break;
+    case UW_PIPE_EXPONENT:
+      if ((st = launch_decode(m, 1, scratch, status, s)) != UW_OK) return st;
+      a.loader = kLoaderEXP8;
+      a.sm = m->sm;
+      a.aux = static_cast<const uint8_t*>(scratch);
+      break;
+    case UW_PIPE_TRANSCODE:
+    case UW_PIPE_DIRECT: {
+      const uint8_t* idx4 = m->idx4;
+      if (pipeline == UW_PIPE_TRANSCODE) {
+        if ((st = launch_decode(m, 2, scratch, status, s)) != UW_OK) return st;
+        idx4 = static_cast<const uint8_t*>(scratch);
+      }
+      if (!idx4) return UW_ERR_INVALID_ARG;
+      a.loader = kLoaderIDX4;
+      a.sm = m->sm;
+      a.aux = idx4;
+      a.vflags = m->vflags;
+      a.vprefix = m->vprefix;
+      a.verbatim = m->verbatim;
+      a.palette = m->cb.palette;
+      a.code_len = m->cb.code_len;
+      break;
+    }
+  }
+  return launch_gemm(a, s);
+}
+
+int sm_count_or_default() {
+  DeviceInfo dev;
+  return device_info(&dev) == UW_OK ? dev.sm_count : 148;
+}
+
+}  // namespace
+
+extern "C" uw_status uw_gemm(const uw_matrix* m, int32_t pipeline, const uint16_t* x, int32_t batch, uint16_t* y,
+                             void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !ws) return UW_ERR_INVALID_ARG;
+  if (pipeline < UW_PIPE_FULL || pipeline > UW_PIPE_DIRECT) return UW_ERR_INVALID_ARG;
+  GemmPlan plan;
+  uw_status st = gemm_plan(m->L.rows, m->L.cols, batch, sm_count_or_default(), &plan);
+  if (st != UW_OK) return st;
+  const size_t base = gemm_ws_bytes(plan);
+  const size_t scratch = pipeline_scratch_bytes(&m->L, pipeline);
+  if (ws_bytes < base + scratch) return UW_ERR_WORKSPACE_TOO_SMALL;
+  return run_pipeline(m, pipeline, x, batch, y, nullptr, ws, base, static_cast<uint8_t*>(ws) + base, scratch,
+                      static_cast<cudaStream_t>(stream));
+}
+
+extern "C" uw_status uw_gemm_direct_palette(const uw_matrix* m, const uint16_t* x, int32_t batch, uint16_t* y,
+                                            void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !m->idx4) return UW_ERR_INVALID_ARG;
+  return uw_gemm(m, UW_PIPE_DIRECT, x, batch, y, ws, ws_bytes, stream);
+}
+
+extern "C" uw_status uw_gemm_direct_palette_general_lookup(const uw_matrix* m, const uint16_t* x, int32_t batch,
+                                                           uint16_t* y, void* ws, size_t ws_bytes, void* stream) {
+  if (!m || !m->idx4 || !ws) return UW_ERR_INVALID_ARG;
+  return run_pipeline(m, UW_PIPE_DIRECT, x, batch, y, nullptr, ws, ws_bytes, nullptr, 0,
+                      static_cast<cudaStream_t>(stream), 1);
+}
+
+extern "C" uw_status uw_gemm_bf16(const uint16_t* w, int64_t rows, int64_t cols, const uint16_t* x, int32_t batch,
+                                  uint16_t* y, void* ws, size_t ws_bytes, void* stream) {
+  GemmArgs a;
+  a.loader = kLoaderBF16;
+  a.N = rows;
+  a.K = cols;
+  a.B = batch;
+  a.wbf16 = w;
+  a.x = x;
+  a.y = y;
+  a.ws = ws;
+  a.ws_bytes = ws_bytes;
+  return launch_gemm(a, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" uw_status uw_swiglu(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t n, void* stream) {
+  return launch_swiglu(g, u, h, n, static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+struct MlpWs {
+  size_t gemm = 0, scratch = 0, gbuf = 0, hbuf = 0, total = 0;
+};
+bool mlp_ws(const uw_matrix* gate, const uw_matrix* up, const uw_matrix* down, const int32_t* pipes, int32_t batch,
+            MlpWs* out) {
+  if (!gate || !up || !down || !pipes) return false;
+  const int64_t ffn = gate->L.rows, d = gate->L.cols;
+  if (up->L.rows != ffn || up->L.cols != d || down->L.rows != d || down->L.cols != ffn) return false;
+  const int sms = sm_count_or_default();
+  MlpWs w;
+  const uw_matrix* ms[3] = {gate, up, down};
+  for (int i = 0; i < 3; ++i) {
+    if (pipes[i] < UW_PIPE_FULL || pipes[i] > UW_PIPE_DIRECT) return false;
+    GemmPlan p;
+    if (gemm_plan(ms[i]->L.rows, ms[i]->L.cols, batch, sms, &p) != UW_OK) return false;
+    w.gemm = std::max(w.gemm, gemm_ws_bytes(p));
+    w.scratch = std::max(w.scratch, pipeline_scratch_bytes(&ms[i]->L, pipes[i]));
+  }
+  w.gbuf = align_up(static_cast<size_t>(batch) * ffn * 2, 256);
+  w.hbuf = w.gbuf;
+  w.total = w.gemm + w.scratch + w.gbuf + w.hbuf;
+  *out = w;
+  return true;
+}
+}  // namespace
+
+extern "C" size_t uw_mlp_workspace_bytes(const uw_matrix* gate, const uw_matrix* up, const uw_matrix* down,
+                                         const int32_t* pipelines, int32_t batch) {
+  MlpWs w;
+  return mlp_ws(gate, up, down, pipelines, batch, &w) ? w.total : 0;
+}
+
+extern "C" uw_status uw_mlp_block(const uw_matrix* gate, const uw_matrix* up, const uw_matrix* down,
+                                  const int32_t* pipelines, const uint16_t* x, int32_t batch, uint16_t* y,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  MlpWs w;
+  if (!ws || !x || !y) return UW_ERR_INVALID_ARG;
+  if (!mlp_ws(gate, up, down, pipelines, batch, &w)) return UW_ERR_INVALID_ARG;
+  if (ws_bytes < w.total) return UW_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  void* scratch = base + w.gemm;
+  uint16_t* g = reinterpret_cast<uint16_t*>(base + w.gemm + w.scratch);
+  uint16_t* h = reinterpret_cast<uint16_t*>(base + w.gemm + w.scratch + w.gbuf);
+  uw_status st = run_pipeline(gate, pipelines[0], x, batch, g, nullptr, ws, w.gemm, scratch, w.scratch, s);
+  if (st != UW_OK) return st;
+  st = run_pipeline(up, pipelines[1], x, batch, h, g, ws, w.gemm, scratch, w.scratch, s);
+  if (st != UW_OK) return st;
+  return run_pipeline(down, pipelines[2], h, batch, y, nullptr, ws, w.gemm, scratch, w.scratch, s);
+}

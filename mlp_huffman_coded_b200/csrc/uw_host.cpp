@@ -1,0 +1,329 @@
+// Host half of libuw: palette + canonical Huffman codebook, the offline
+// encoder and the host-side format validator.
+//
+// Method: Cloudflare, "Unweight: how we compressed an LLM 22% without
+// sacrificing quality", section "How to compress model weights effectively"
+// (raw sign/mantissa, Huffman-coded exponent against a top-16 palette,
+// verbatim 64-element rows).  The storage layout is documented in uw.h.
+#include <algorithm>
+#include <array>
+#include <cstdint>
+#include <cstring>
+#include <queue>
+#include <utility>
+#include <vector>
+
+#include "uw.h"
+
+namespace {
+
+constexpr int kGroup = UW_GROUP;
+constexpr int kPal = UW_PALETTE;
+
+inline int popc32(uint32_t v) { return __builtin_popcount(v); }
+
+bool shape_ok(int64_t rows, int64_t cols) {
+  return rows >= 1 && cols >= kGroup && cols % kGroup == 0 && rows <= (int64_t(1) << 40) / cols;
+}
+
+// exponent value -> palette index, 255 when outside the palette
+std::array<uint8_t, 256> palette_map(const uint8_t* palette) {
+  std::array<uint8_t, 256> m;
+  m.fill(255);
+  for (int i = 0; i < kPal; ++i) m[palette[i]] = static_cast<uint8_t>(i);
+  return m;
+}
+
+// Code lengths by the two-smallest-merge construction.  Ties between equal
+// weights go to the smaller node id; leaves are the palette indices 0..15 and
+// merged nodes are numbered 16, 17, ... in creation order.
+void huffman_lengths(const uint64_t* freq, uint8_t* len_out) {
+  std::memset(len_out, 0, kPal);
+  using Node = std::pair<uint64_t, int>;  // (weight, id)
+  std::priority_queue<Node, std::vector<Node>, std::greater<Node>> heap;
+  int used = 0, only = -1;
+  for (int i = 0; i < kPal; ++i)
+    if (freq[i] > 0) {
+      heap.push({freq[i], i});
+      ++used;
+      only = i;
+    }
+  if (used == 0) return;
+  if (used == 1) {
+    len_out[only] = 1;
+    return;
+  }
+  std::vector<int> parent(2 * kPal, -1);
+  int next_id = kPal;
+  while (heap.size() > 1) {
+    Node a = heap.top();
+    heap.pop();
+    Node b = heap.top();
+    heap.pop();
+    parent[a.second] = next_id;
+    parent[b.second] = next_id;
+    heap.push({a.first + b.first, next_id});
+    ++next_id;
+  }
+  for (int i = 0; i < kPal; ++i) {
+    if (freq[i] == 0) continue;
+    int d = 0;
+    for (int n = i; parent[n] >= 0; n = parent[n]) ++d;
+    len_out[i] = static_cast<uint8_t>(d);
+  }
+}
+
+// Canonical codes: (length, index) order, consecutive values, shifted left
+// whenever the length grows.
+void canonical(const uint8_t* len, uint16_t* code) {
+  std::vector<std::pair<int, int>> order;
+  for (int i = 0; i < kPal; ++i) {
+    code[i] = 0;
+    if (len[i]) order.push_back({len[i], i});
+  }
+  std::sort(order.begin(), order.end());
+  uint32_t c = 0;
+  int prev = order.empty() ? 0 : order[0].first;
+  for (auto& li : order) {
+    c <<= (li.first - prev);
+    code[li.second] = static_cast<uint16_t>(c);
+    ++c;
+    prev = li.first;
+  }
+}
+
+}  // namespace
+
+extern "C" uw_status uw_build_palette_codebook(const uint16_t* w, int64_t rows, int64_t cols,
+                                                uw_codebook* out) {
+  if (!w || !out) return UW_ERR_INVALID_ARG;
+  if (!shape_ok(rows, cols)) return UW_ERR_UNSUPPORTED_SHAPE;
+  const int64_t n = rows * cols;
+  std::array<uint64_t, 256> hist{};
+  for (int64_t i = 0; i < n; ++i) ++hist[(w[i] >> 7) & 0xFF];
+  std::array<int, 256> order;
+  for (int e = 0; e < 256; ++e) order[e] = e;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+    if (hist[a] != hist[b]) return hist[a] > hist[b];
+    return a < b;
+  });
+  uw_codebook cb;
+  std::memset(&cb, 0, sizeof(cb));
+  for (int i = 0; i < kPal; ++i) cb.palette[i] = static_cast<uint8_t>(order[i]);
+  auto pm = palette_map(cb.palette);
+  // frequencies over non-verbatim groups only
+  const int64_t n_groups = n / kGroup;
+  for (int64_t g = 0; g < n_groups; ++g) {
+    const uint16_t* p = w + g * kGroup;
+    bool verb = false;
+    for (int k = 0; k < kGroup; ++k) verb |= pm[(p[k] >> 7) & 0xFF] == 255;
+    if (verb) continue;
+    for (int k = 0; k < kGroup; ++k) ++cb.freq[pm[(p[k] >> 7) & 0xFF]];
+  }
+  huffman_lengths(cb.freq, cb.code_len);
+  canonical(cb.code_len, cb.code);
+  int ns = 0, ml = 0;
+  for (int i = 0; i < kPal; ++i) {
+    ns += cb.code_len[i] > 0;
+    ml = std::max<int>(ml, cb.code_len[i]);
+  }
+  cb.n_symbols = static_cast<uint8_t>(ns);
+  cb.max_len = static_cast<uint8_t>(ml);
+  *out = cb;
+  return UW_OK;
+}
+
+extern "C" uw_status uw_encode(const uint16_t* w, int64_t rows, int64_t cols, const uw_codebook* cb,
+                               int32_t chunk_groups, uw_layout* L, uint8_t* sm, uint32_t* stream,
+                               uint32_t* chunk_bit_off, uint32_t* vflags, uint32_t* vprefix,
+                               uint16_t* verbatim) {
+  if (!w || !cb || !L) return UW_ERR_INVALID_ARG;
+  if (!shape_ok(rows, cols) || chunk_groups < 1 || chunk_groups > 16) return UW_ERR_UNSUPPORTED_SHAPE;
+  for (int i = 0; i < kPal; ++i)
+    if (cb->code_len[i] > UW_MAX_CODE_LEN) return UW_ERR_CORRUPT;
+  const int64_t gpr = cols / kGroup;
+  const int64_t n_groups = rows * gpr;
+  const int32_t wpr = static_cast<int32_t>((gpr + 31) / 32);
+  auto pm = palette_map(cb->palette);
+
+  // pass 1: verbatim flags and coded bits per group
+  std::vector<uint8_t> verb(n_groups);
+  std::vector<uint32_t> gbits(n_groups);
+  uint64_t total = 0;
+  int64_t n_verb = 0;
+  for (int64_t g = 0; g < n_groups; ++g) {
+    const uint16_t* p = w + g * kGroup;
+    bool v = false;
+    for (int k = 0; k < kGroup; ++k) v |= pm[(p[k] >> 7) & 0xFF] == 255;
+    verb[g] = v;
+    uint32_t b = 0;
+    if (!v) {
+      for (int k = 0; k < kGroup; ++k) {
+        uint8_t len = cb->code_len[pm[(p[k] >> 7) & 0xFF]];
+        if (len == 0) return UW_ERR_CORRUPT;
+        b += len;
+      }
+    } else {
+      ++n_verb;
+    }
+    gbits[g] = b;
+    total += b;
+  }
+  if (total >= (uint64_t(1) << 32)) return UW_ERR_UNSUPPORTED_SHAPE;
+
+  uw_layout lay;
+  std::memset(&lay, 0, sizeof(lay));
+  lay.rows = rows;
+  lay.cols = cols;
+  lay.chunk_groups = chunk_groups;
+  lay.words_per_row = wpr;
+  lay.n_groups = n_groups;
+  lay.n_chunks = (n_groups + chunk_groups - 1) / chunk_groups;
+  lay.n_verbatim = n_verb;
+  lay.total_bits = static_cast<int64_t>(total);
+  lay.stream_words = static_cast<int64_t>((total + 31) / 32) + 2;
+  *L = lay;
+  if (!sm && !stream && !chunk_bit_off && !vflags && !vprefix && !verbatim) return UW_OK;
+  if (!sm || !stream || !chunk_bit_off || !vflags || !vprefix || (n_verb > 0 && !verbatim))
+    return UW_ERR_INVALID_ARG;
+
+  // sign+mantissa bytes: own mantissa, pair partner's sign
+  const int64_t n = rows * cols;
+  for (int64_t i = 0; i < n; i += 2) {
+    uint16_t a = w[i], b = w[i + 1];
+    sm[i] = static_cast<uint8_t>(((a & 0x7F) << 1) | (b >> 15));
+    sm[i + 1] = static_cast<uint8_t>(((b & 0x7F) << 1) | (a >> 15));
+  }
+
+  // chunk offsets
+  uint64_t pos = 0;
+  for (int64_t g = 0; g < n_groups; ++g) {
+    if (g % chunk_groups == 0) chunk_bit_off[g / chunk_groups] = static_cast<uint32_t>(pos);
+    pos += gbits[g];
+  }
+  chunk_bit_off[lay.n_chunks] = static_cast<uint32_t>(pos);
+
+  // bitstream, MSB first
+  std::memset(stream, 0, lay.stream_words * sizeof(uint32_t));
+  uint64_t acc = 0;  // pending bits, right aligned
+  int nacc = 0;
+  int64_t wi = 0;
+  for (int64_t g = 0; g < n_groups; ++g) {
+    if (verb[g]) continue;
+    const uint16_t* p = w + g * kGroup;
+    for (int k = 0; k < kGroup; ++k) {
+      int s = pm[(p[k] >> 7) & 0xFF];
+      acc = (acc << cb->code_len[s]) | cb->code[s];
+      nacc += cb->code_len[s];
+      if (nacc >= 32) {
+        stream[wi++] = static_cast<uint32_t>(acc >> (nacc - 32));
+        nacc -= 32;
+        acc &= (uint64_t(1) << nacc) - 1;
+      }
+    }
+  }
+  if (nacc > 0) stream[wi++] = static_cast<uint32_t>(acc << (32 - nacc));
+
+  // verbatim flags, per-word prefix counts, verbatim store
+  std::memset(vflags, 0, sizeof(uint32_t) * rows * wpr);
+  for (int64_t g = 0; g < n_groups; ++g)
+    if (verb[g]) {
+      int64_t r = g / gpr, j = g % gpr;
+      vflags[r * wpr + j / 32] |= 1u << (j % 32);
+    }
+  uint32_t run = 0;
+  for (int64_t i = 0; i < rows * wpr; ++i) {
+    vprefix[i] = run;
+    run += popc32(vflags[i]);
+  }
+  vprefix[rows * wpr] = run;
+  int64_t vs = 0;
+  for (int64_t g = 0; g < n_groups; ++g)
+    if (verb[g]) std::memcpy(verbatim + (vs++) * kGroup, w + g * kGroup, kGroup * sizeof(uint16_t));
+  return UW_OK;
+}
+
+extern "C" uw_status uw_validate(const uw_matrix* m) {
+  if (!m) return UW_ERR_INVALID_ARG;
+  const uw_layout& L = m->L;
+  if (!shape_ok(L.rows, L.cols) || L.chunk_groups < 1 || L.chunk_groups > 16)
+    return UW_ERR_UNSUPPORTED_SHAPE;
+  const int64_t gpr = L.cols / kGroup;
+  if (L.n_groups != L.rows * gpr || L.words_per_row != (gpr + 31) / 32 ||
+      L.n_chunks != (L.n_groups + L.chunk_groups - 1) / L.chunk_groups ||
+      L.stream_words != (L.total_bits + 31) / 32 + 2 || L.total_bits < 0 ||
+      L.total_bits >= (int64_t(1) << 32))
+    return UW_ERR_CORRUPT;
+  if (!m->sm || !m->stream || !m->chunk_bit_off || !m->vflags || !m->vprefix ||
+      (L.n_verbatim > 0 && !m->verbatim))
+    return UW_ERR_INVALID_ARG;
+  // codebook: lengths <= 15, Kraft sum <= 1, codes canonical for the lengths
+  const uw_codebook& cb = m->cb;
+  uint64_t kraft = 0;  // in units of 2^-15
+  int ns = 0, ml = 0;
+  for (int i = 0; i < kPal; ++i) {
+    if (cb.code_len[i] > UW_MAX_CODE_LEN) return UW_ERR_CORRUPT;
+    if (cb.code_len[i]) {
+      kraft += uint64_t(1) << (UW_MAX_CODE_LEN - cb.code_len[i]);
+      ++ns;
+      ml = std::max<int>(ml, cb.code_len[i]);
+    }
+  }
+  if (kraft > (uint64_t(1) << UW_MAX_CODE_LEN)) return UW_ERR_CORRUPT;
+  if (cb.n_symbols != ns || cb.max_len != ml) return UW_ERR_CORRUPT;
+  uint16_t expect[kPal];
+  canonical(cb.code_len, expect);
+  for (int i = 0; i < kPal; ++i)
+    if (cb.code_len[i] && cb.code[i] != expect[i]) return UW_ERR_CORRUPT;
+  for (int i = 0; i < kPal; ++i)
+    for (int j = i + 1; j < kPal; ++j)
+      if (cb.palette[i] == cb.palette[j]) return UW_ERR_CORRUPT;
+  // offsets monotone, ending at total_bits; groups of a chunk need at least
+  // 64 * (shortest code) bits unless verbatim -- checked loosely as monotone
+  if (m->chunk_bit_off[0] != 0) return UW_ERR_CORRUPT;
+  for (int64_t c = 0; c < L.n_chunks; ++c)
+    if (m->chunk_bit_off[c + 1] < m->chunk_bit_off[c]) return UW_ERR_CORRUPT;
+  if (int64_t(m->chunk_bit_off[L.n_chunks]) != L.total_bits) return UW_ERR_CORRUPT;
+  // flag words: no bits beyond the row's groups; prefix = running popcount
+  const int64_t nw = L.rows * L.words_per_row;
+  uint32_t run = 0;
+  for (int64_t i = 0; i < nw; ++i) {
+    int64_t j = i % L.words_per_row;
+    int64_t valid = std::min<int64_t>(32, gpr - 32 * j);
+    if (valid < 32 && (m->vflags[i] >> valid) != 0) return UW_ERR_CORRUPT;
+    if (m->vprefix[i] != run) return UW_ERR_CORRUPT;
+    run += popc32(m->vflags[i]);
+  }
+  if (m->vprefix[nw] != run || int64_t(run) != L.n_verbatim) return UW_ERR_CORRUPT;
+  // a chunk's coded groups need between 64*min_len and 64*max_len bits each
+  int minl = 16;
+  for (int i = 0; i < kPal; ++i)
+    if (cb.code_len[i]) minl = std::min<int>(minl, cb.code_len[i]);
+  for (int64_t c = 0; c < L.n_chunks; ++c) {
+    int64_t coded = 0;
+    for (int64_t g = c * L.chunk_groups; g < std::min<int64_t>((c + 1) * L.chunk_groups, L.n_groups); ++g) {
+      int64_t r = g / gpr, j = g % gpr;
+      coded += !((m->vflags[r * L.words_per_row + j / 32] >> (j % 32)) & 1);
+    }
+    int64_t bits = int64_t(m->chunk_bit_off[c + 1]) - m->chunk_bit_off[c];
+    if (coded == 0 ? bits != 0 : (ns == 0 || bits < coded * kGroup * minl || bits > coded * kGroup * ml))
+      return UW_ERR_CORRUPT;
+  }
+  return UW_OK;
+}
+
+extern "C" const char* uw_status_string(uw_status s) {
+  switch (s) {
+    case UW_OK: return "ok";
+    case UW_ERR_INVALID_ARG: return "invalid argument";
+    case UW_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case UW_ERR_CORRUPT: return "corrupt compressed data";
+    case UW_ERR_TIMEOUT: return "on-GPU wait timed out";
+    case UW_ERR_CUDA: return "CUDA error";
+    case UW_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case UW_ERR_NO_DEVICE: return "no sm_100 device";
+  }
+  return "unknown status";
+}
+
+extern "C" int32_t uw_version(void) { return 100; }

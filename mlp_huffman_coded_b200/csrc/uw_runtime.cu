@@ -1,0 +1,182 @@
+// Host runtime of libuw: device facts, tensor-map creation, workspace
+// management, argument checks and the public decode entry points.
+#include <atomic>
+#include <cstring>
+#include <mutex>
+
+#include "uw_internal.h"
+
+namespace uw {
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+std::mutex g_dev_mu;
+DeviceInfo g_dev_cache[64];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+}  // namespace
+
+void note_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
+uw_status device_info(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return UW_ERR_NO_DEVICE;
+  }
+  if (dev < 0 || dev >= 64) return UW_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev_cache[dev];
+  if (d.ordinal != dev) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return UW_ERR_NO_DEVICE;
+    }
+    d.ordinal = dev;
+    d.sm_count = prop.multiProcessorCount;
+    d.major = prop.major;
+    d.minor = prop.minor;
+    d.max_smem_optin = prop.sharedMemPerBlockOptin;
+    d.l2_bytes = prop.l2CacheSize;
+  }
+  if (d.major != 10) return UW_ERR_NO_DEVICE;
+  *out = d;
+  return UW_OK;
+}
+
+uw_status make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                             uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                             uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    else
+      cudaGetLastError();
+  });
+  if (!g_encode) return UW_ERR_CUDA;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? UW_OK : UW_ERR_CUDA;
+}
+
+uw_status check_matrix(const uw_matrix* m) {
+  if (!m) return UW_ERR_INVALID_ARG;
+  const uw_layout& L = m->L;
+  if (L.rows < 1 || L.cols < 64 || L.cols % 64 != 0) return UW_ERR_UNSUPPORTED_SHAPE;
+  if (L.chunk_groups < 1 || L.chunk_groups > 16) return UW_ERR_UNSUPPORTED_SHAPE;
+  const int64_t gpr = L.cols / 64;
+  if (L.n_groups != L.rows * gpr || L.words_per_row != (gpr + 31) / 32 ||
+      L.n_chunks != (L.n_groups + L.chunk_groups - 1) / L.chunk_groups || L.stream_words < 2 ||
+      L.n_verbatim < 0 || L.n_verbatim > L.n_groups)
+    return UW_ERR_CORRUPT;
+  if (m->cb.max_len > UW_MAX_CODE_LEN) return UW_ERR_CORRUPT;
+  if (!m->sm || !m->stream || !m->chunk_bit_off || !m->vflags || !m->vprefix) return UW_ERR_INVALID_ARG;
+  if (L.n_verbatim > 0 && !m->verbatim) return UW_ERR_INVALID_ARG;
+  if (!aligned16(m->sm) || !aligned16(m->stream) || !aligned16(m->chunk_bit_off) || !aligned16(m->vflags) ||
+      !aligned16(m->vprefix) || (m->verbatim && !aligned16(m->verbatim)) || (m->idx4 && !aligned16(m->idx4)))
+    return UW_ERR_INVALID_ARG;
+  return UW_OK;
+}
+
+uw_status gemm_plan(int64_t N, int64_t K, int B, int sm_count, GemmPlan* out) {
+  if (N < 1 || K < 64 || K % 64 != 0) return UW_ERR_UNSUPPORTED_SHAPE;
+  if (B < 1 || B > UW_MAX_BATCH) return UW_ERR_UNSUPPORTED_SHAPE;
+  if (K > 32768) return UW_ERR_UNSUPPORTED_SHAPE;  // per-tile flag words are staged on chip
+  if (N > (int64_t(1) << 31) - 128) return UW_ERR_UNSUPPORTED_SHAPE;
+  GemmPlan p;
+  p.N = N;
+  p.K = K;
+  p.B = B;
+  p.KB = static_cast<int>(K / 64);
+  p.n_mtiles = static_cast<int>((N + 127) / 128);
+  p.n_ntiles = (B + 255) / 256;
+  const int per = (B + p.n_ntiles - 1) / p.n_ntiles;
+  p.ntile = (per + 15) / 16 * 16;
+  p.units = static_cast<int64_t>(p.n_mtiles) * p.n_ntiles * p.KB;
+  p.grid = static_cast<int>(p.units < sm_count ? p.units : sm_count);
+  const int64_t n_tiles = static_cast<int64_t>(p.n_mtiles) * p.n_ntiles;
+  p.counter_bytes = align_up(static_cast<size_t>(n_tiles) * 4, 256);
+  p.partial_bytes = static_cast<size_t>(n_tiles + p.grid) * p.ntile * 128 * 4;
+  *out = p;
+  return UW_OK;
+}
+
+size_t gemm_ws_bytes(const GemmPlan& p) { return kWsHeader + p.counter_bytes + align_up(p.partial_bytes, 256); }
+
+size_t pipeline_scratch_bytes(const uw_layout* L, int pipeline) {
+  const size_t n = static_cast<size_t>(L->rows) * static_cast<size_t>(L->cols);
+  switch (pipeline) {
+    case UW_PIPE_FULL: return align_up(n * 2, 256);
+    case UW_PIPE_EXPONENT: return align_up(n, 256);
+    case UW_PIPE_TRANSCODE: return align_up(n / 2, 256);
+    default: return 0;
+  }
+}
+
+}  // namespace uw
+
+using namespace uw;
+
+extern "C" size_t uw_workspace_bytes(const uw_layout* L, int32_t pipeline, int32_t batch) {
+  if (!L || pipeline < 0 || pipeline > UW_PIPE_BF16) return 0;
+  if (batch == 0) return kWsHeader;
+  DeviceInfo dev;
+  const int sms = device_info(&dev) == UW_OK ? dev.sm_count : 148;
+  GemmPlan p;
+  if (gemm_plan(L->rows, L->cols, batch, sms, &p) != UW_OK) return 0;
+  return gemm_ws_bytes(p) + pipeline_scratch_bytes(L, pipeline);
+}
+
+extern "C" uw_status uw_workspace_init(void* ws, size_t bytes, void* stream) {
+  if (!ws || bytes < kWsHeader || !aligned16(ws)) return UW_ERR_INVALID_ARG;
+  return cuda_status(cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream)));
+}
+
+extern "C" uw_status uw_workspace_status(void* ws, void* stream) {
+  if (!ws) return UW_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return UW_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return UW_ERR_CUDA;
+  if (v != 0) {
+    if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return UW_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return UW_ERR_CUDA;
+  }
+  return static_cast<uw_status>(v);
+}
+
+static uw_status decode_entry(const uw_matrix* m, int mode, void* out, void* ws, size_t ws_bytes,
+                              void* stream) {
+  if (!ws || ws_bytes < kWsHeader || !aligned16(ws)) return ws ? UW_ERR_WORKSPACE_TOO_SMALL : UW_ERR_INVALID_ARG;
+  return launch_decode(m, mode, out, static_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream));
+}
+
+extern "C" uw_status uw_decode_full(const uw_matrix* m, uint16_t* out, void* ws, size_t ws_bytes, void* stream) {
+  return decode_entry(m, 0, out, ws, ws_bytes, stream);
+}
+
+extern "C" uw_status uw_decode_exponent_only(const uw_matrix* m, uint8_t* out, void* ws, size_t ws_bytes,
+                                             void* stream) {
+  return decode_entry(m, 1, out, ws, ws_bytes, stream);
+}
+
+extern "C" uw_status uw_transcode_palette(const uw_matrix* m, uint8_t* out, void* ws, size_t ws_bytes,
+                                          void* stream) {
+  return decode_entry(m, 2, out, ws, ws_bytes, stream);
+}
+
+extern "C" uint64_t uw_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -1,0 +1,349 @@
+"""Thin ctypes binding of libuw (include/uw.h).
+
+Argument marshalling only: every step of the compressed-weight path runs in
+the C++ host codec or the CUDA kernels of libuw.so.  PyTorch is used for
+device memory (``tensor.data_ptr()``) and streams
+(``torch.cuda.current_stream().cuda_stream``) and nothing else.
+
+``lib()`` raises ``UwError`` when the library has not been built; there is no
+fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libuw.so")
+
+PIPE_FULL, PIPE_EXPONENT, PIPE_TRANSCODE, PIPE_DIRECT, PIPE_BF16 = 0, 1, 2, 3, 4
+PIPELINES = {"full": PIPE_FULL, "exponent": PIPE_EXPONENT, "transcode": PIPE_TRANSCODE,
+             "direct": PIPE_DIRECT}
+PIPE_NAMES = {v: k for k, v in PIPELINES.items()}
+PIPE_NAMES[PIPE_BF16] = "bf16"
+
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "corrupt compressed data",
+          4: "on-GPU wait timed out", 5: "CUDA error", 6: "workspace too small", 7: "no sm_100 device"}
+UW_OK, UW_ERR_INVALID_ARG, UW_ERR_UNSUPPORTED_SHAPE, UW_ERR_CORRUPT = 0, 1, 2, 3
+UW_ERR_TIMEOUT, UW_ERR_CUDA, UW_ERR_WORKSPACE_TOO_SMALL, UW_ERR_NO_DEVICE = 4, 5, 6, 7
+
+
+class UwError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = int(status)
+        super().__init__(f"{what}: {STATUS.get(int(status), 'status %d' % status)} ({int(status)})")
+
+
+class Codebook(C.Structure):
+    _fields_ = [("palette", C.c_uint8 * 16), ("code_len", C.c_uint8 * 16), ("code", C.c_uint16 * 16),
+                ("freq", C.c_uint64 * 16), ("n_symbols", C.c_uint8), ("max_len", C.c_uint8),
+                ("reserved", C.c_uint8 * 6)]
+
+
+class Layout(C.Structure):
+    _fields_ = [("rows", C.c_int64), ("cols", C.c_int64), ("chunk_groups", C.c_int32),
+                ("words_per_row", C.c_int32), ("n_groups", C.c_int64), ("n_chunks", C.c_int64),
+                ("n_verbatim", C.c_int64), ("stream_words", C.c_int64), ("total_bits", C.c_int64)]
+
+
+class Matrix(C.Structure):
+    _fields_ = [("L", Layout), ("cb", Codebook), ("sm", C.c_void_p), ("stream", C.c_void_p),
+                ("chunk_bit_off", C.c_void_p), ("vflags", C.c_void_p), ("vprefix", C.c_void_p),
+                ("verbatim", C.c_void_p), ("idx4", C.c_void_p)]
+
+
+_P = C.c_void_p
+_SIGS = {
+    "uw_build_palette_codebook": (C.c_int, [_P, C.c_int64, C.c_int64, C.POINTER(Codebook)]),
+    "uw_encode": (C.c_int, [_P, C.c_int64, C.c_int64, C.POINTER(Codebook), C.c_int32, C.POINTER(Layout),
+                            _P, _P, _P, _P, _P, _P]),
+    "uw_validate": (C.c_int, [C.POINTER(Matrix)]),
+    "uw_workspace_bytes": (C.c_size_t, [C.POINTER(Layout), C.c_int32, C.c_int32]),
+    "uw_workspace_init": (C.c_int, [_P, C.c_size_t, _P]),
+    "uw_workspace_status": (C.c_int, [_P, _P]),
+    "uw_decode_full": (C.c_int, [C.POINTER(Matrix), _P, _P, C.c_size_t, _P]),
+    "uw_decode_exponent_only": (C.c_int, [C.POINTER(Matrix), _P, _P, C.c_size_t, _P]),
+    "uw_transcode_palette": (C.c_int, [C.POINTER(Matrix), _P, _P, C.c_size_t, _P]),
+    "uw_gemm_direct_palette": (C.c_int, [C.POINTER(Matrix), _P, C.c_int32, _P, _P, C.c_size_t, _P]),
+    "uw_gemm_direct_palette_general_lookup": (C.c_int, [C.POINTER(Matrix), _P, C.c_int32, _P, _P,
+                                                        C.c_size_t, _P]),
+    "uw_gemm": (C.c_int, [C.POINTER(Matrix), C.c_int32, _P, C.c_int32, _P, _P, C.c_size_t, _P]),
+    "uw_gemm_bf16": (C.c_int, [_P, C.c_int64, C.c_int64, _P, C.c_int32, _P, _P, C.c_size_t, _P]),
+    "uw_swiglu": (C.c_int, [_P, _P, _P, C.c_int64, _P]),
+    "uw_mlp_workspace_bytes": (C.c_size_t, [C.POINTER(Matrix), C.POINTER(Matrix), C.POINTER(Matrix),
+                                            C.POINTER(C.c_int32), C.c_int32]),
+    "uw_mlp_block": (C.c_int, [C.POINTER(Matrix), C.POINTER(Matrix), C.POINTER(Matrix), C.POINTER(C.c_int32),
+                               _P, C.c_int32, _P, _P, C.c_size_t, _P]),
+    "uw_autotune": (C.c_int, [C.POINTER(Matrix), C.POINTER(C.c_int32), C.c_int32, C.c_int32, _P, _P, _P,
+                              C.c_size_t, _P, C.c_size_t, C.POINTER(C.c_int32), C.POINTER(C.c_float), _P]),
+    "uw_status_string": (C.c_char_p, [C.c_int]),
+    "uw_version": (C.c_int32, []),
+    "uw_launch_count": (C.c_uint64, []),
+}
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load libuw.so (built by ``python -m mlp_huffman_coded_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise UwError(UW_ERR_NO_DEVICE, f"libuw.so not built at {LIB_PATH}")
+        h = C.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(h, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = h
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != UW_OK:
+        raise UwError(status, what)
+
+
+def _ptr(a) -> int:
+    """Address of a numpy array or torch tensor (None -> NULL)."""
+    if a is None:
+        return None
+    if isinstance(a, np.ndarray):
+        return a.ctypes.data
+    return a.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+# ---------------------------------------------------------------------------
+# host codec
+# ---------------------------------------------------------------------------
+
+@dataclass
+class HostEncoded:
+    layout: Layout
+    cb: Codebook
+    sm: np.ndarray
+    stream: np.ndarray
+    chunk_bit_off: np.ndarray
+    vflags: np.ndarray
+    vprefix: np.ndarray
+    verbatim: np.ndarray
+
+    @property
+    def rows(self):
+        return int(self.layout.rows)
+
+    @property
+    def cols(self):
+        return int(self.layout.cols)
+
+    def matrix(self) -> Matrix:
+        """uw_matrix whose pointers are these host arrays (for uw_validate)."""
+        m = Matrix()
+        m.L = self.layout
+        m.cb = self.cb
+        m.sm, m.stream, m.chunk_bit_off = _ptr(self.sm), _ptr(self.stream), _ptr(self.chunk_bit_off)
+        m.vflags, m.vprefix = _ptr(self.vflags), _ptr(self.vprefix)
+        m.verbatim = _ptr(self.verbatim) if self.verbatim.size else None
+        m.idx4 = None
+        return m
+
+    def compressed_bytes(self, form: str = "huffman") -> int:
+        meta = self.vflags.nbytes + self.vprefix.nbytes + self.verbatim.nbytes
+        if form == "huffman":
+            return self.sm.nbytes + self.stream.nbytes + self.chunk_bit_off.nbytes + meta
+        if form == "palette":
+            return self.sm.nbytes + self.rows * self.cols // 2 + meta
+        raise ValueError(form)
+
+
+def build_codebook(w: np.ndarray) -> Codebook:
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    cb = Codebook()
+    _check(lib().uw_build_palette_codebook(_ptr(w), w.shape[0], w.shape[1], C.byref(cb)),
+           "uw_build_palette_codebook")
+    return cb
+
+
+def encode(w: np.ndarray, chunk_groups: int = 4, cb: Codebook | None = None) -> HostEncoded:
+    w = np.ascontiguousarray(w, dtype=np.uint16)
+    rows, cols = w.shape
+    if cb is None:
+        cb = build_codebook(w)
+    L = Layout()
+    f = lib().uw_encode
+    _check(f(_ptr(w), rows, cols, C.byref(cb), chunk_groups, C.byref(L), None, None, None, None, None, None),
+           "uw_encode (sizes)")
+    sm = np.empty(rows * cols, np.uint8)
+    stream = np.empty(L.stream_words, np.uint32)
+    off = np.empty(L.n_chunks + 1, np.uint32)
+    vflags = np.empty(rows * L.words_per_row, np.uint32)
+    vprefix = np.empty(rows * L.words_per_row + 1, np.uint32)
+    verbatim = np.empty(L.n_verbatim * 64, np.uint16)
+    _check(f(_ptr(w), rows, cols, C.byref(cb), chunk_groups, C.byref(L), _ptr(sm), _ptr(stream), _ptr(off),
+             _ptr(vflags), _ptr(vprefix), _ptr(verbatim) if verbatim.size else None), "uw_encode")
+    return HostEncoded(L, cb, sm, stream, off, vflags, vprefix, verbatim)
+
+
+def validate(enc: HostEncoded) -> int:
+    """Host-side format check; returns the status code (0 = ok)."""
+    m = enc.matrix()
+    return int(lib().uw_validate(C.byref(m)))
+
+
+# ---------------------------------------------------------------------------
+# device side
+# ---------------------------------------------------------------------------
+
+class Workspace:
+    """Caller-owned device workspace (a torch uint8 tensor), zeroed once."""
+
+    def __init__(self, nbytes: int, device="cuda"):
+        import torch
+        self.nbytes = max(int(nbytes), 256)
+        self.t = torch.zeros(self.nbytes, dtype=torch.uint8, device=device)
+
+    @property
+    def ptr(self) -> int:
+        return self.t.data_ptr()
+
+    def status(self, stream=None) -> int:
+        return int(lib().uw_workspace_status(self.ptr, _stream(stream)))
+
+    def check(self, what="device", stream=None):
+        _check(self.status(stream), what)
+
+
+class DeviceMatrix:
+    """One compressed matrix uploaded to the GPU (torch tensors own memory)."""
+
+    def __init__(self, enc: HostEncoded, device="cuda"):
+        import torch
+
+        def up(a):
+            return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+        self.enc = enc
+        self.device = device
+        self.sm = up(enc.sm)
+        self.stream = up(enc.stream.view(np.int32))
+        self.chunk_bit_off = up(enc.chunk_bit_off.view(np.int32))
+        self.vflags = up(enc.vflags.view(np.int32))
+        self.vprefix = up(enc.vprefix.view(np.int32))
+        self.verbatim = up(enc.verbatim.view(np.int16)) if enc.verbatim.size else None
+        self.idx4 = None
+        self.mat = Matrix()
+        self.mat.L = enc.layout
+        self.mat.cb = enc.cb
+        self.mat.sm, self.mat.stream = self.sm.data_ptr(), self.stream.data_ptr()
+        self.mat.chunk_bit_off = self.chunk_bit_off.data_ptr()
+        self.mat.vflags, self.mat.vprefix = self.vflags.data_ptr(), self.vprefix.data_ptr()
+        self.mat.verbatim = self.verbatim.data_ptr() if self.verbatim is not None else None
+        self.mat.idx4 = None
+
+    @property
+    def rows(self):
+        return self.enc.rows
+
+    @property
+    def cols(self):
+        return self.enc.cols
+
+    def prepare_direct_palette(self, ws: Workspace, stream=None):
+        """Load-time transcode to 4-bit palette indices (direct palette)."""
+        import torch
+        self.idx4 = torch.empty(self.rows * self.cols // 2, dtype=torch.uint8, device=self.device)
+        transcode_palette(self, self.idx4, ws, stream)
+        self.mat.idx4 = self.idx4.data_ptr()
+        return self
+
+    def direct_palette_bytes(self) -> int:
+        """Bytes the direct-palette GEMM reads from HBM for W."""
+        e = self.enc
+        return (e.sm.nbytes + e.rows * e.cols // 2 + e.vflags.nbytes + e.vprefix.nbytes + e.verbatim.nbytes)
+
+
+def workspace_bytes(dm_or_layout, pipeline: int, batch: int) -> int:
+    L = dm_or_layout.mat.L if isinstance(dm_or_layout, DeviceMatrix) else dm_or_layout
+    return int(lib().uw_workspace_bytes(C.byref(L), pipeline, batch))
+
+
+def decode_full(dm: DeviceMatrix, out, ws: Workspace, stream=None):
+    _check(lib().uw_decode_full(C.byref(dm.mat), _ptr(out), ws.ptr, ws.nbytes, _stream(stream)), "uw_decode_full")
+
+
+def decode_exponent_only(dm: DeviceMatrix, out, ws: Workspace, stream=None):
+    _check(lib().uw_decode_exponent_only(C.byref(dm.mat), _ptr(out), ws.ptr, ws.nbytes, _stream(stream)),
+           "uw_decode_exponent_only")
+
+
+def transcode_palette(dm: DeviceMatrix, out, ws: Workspace, stream=None):
+    _check(lib().uw_transcode_palette(C.byref(dm.mat), _ptr(out), ws.ptr, ws.nbytes, _stream(stream)),
+           "uw_transcode_palette")
+
+
+def gemm(dm: DeviceMatrix, pipeline: int, x, y, ws: Workspace, stream=None):
+    _check(lib().uw_gemm(C.byref(dm.mat), pipeline, _ptr(x), x.shape[0], _ptr(y), ws.ptr, ws.nbytes,
+                         _stream(stream)), "uw_gemm")
+
+
+def gemm_direct_palette(dm: DeviceMatrix, x, y, ws: Workspace, stream=None, general_lookup=False):
+    f = lib().uw_gemm_direct_palette_general_lookup if general_lookup else lib().uw_gemm_direct_palette
+    _check(f(C.byref(dm.mat), _ptr(x), x.shape[0], _ptr(y), ws.ptr, ws.nbytes, _stream(stream)),
+           "uw_gemm_direct_palette")
+
+
+def gemm_bf16(w, x, y, ws: Workspace, stream=None):
+    _check(lib().uw_gemm_bf16(_ptr(w), w.shape[0], w.shape[1], _ptr(x), x.shape[0], _ptr(y), ws.ptr, ws.nbytes,
+                              _stream(stream)), "uw_gemm_bf16")
+
+
+def swiglu(g, u, h, stream=None):
+    _check(lib().uw_swiglu(_ptr(g), _ptr(u), _ptr(h), g.numel(), _stream(stream)), "uw_swiglu")
+
+
+def _pipes(pipelines):
+    arr = (C.c_int32 * 3)(*[int(p) for p in pipelines])
+    return arr
+
+
+def mlp_workspace_bytes(gate: DeviceMatrix, up: DeviceMatrix, down: DeviceMatrix, pipelines, batch: int) -> int:
+    return int(lib().uw_mlp_workspace_bytes(C.byref(gate.mat), C.byref(up.mat), C.byref(down.mat),
+                                            _pipes(pipelines), batch))
+
+
+def mlp_block(gate: DeviceMatrix, up: DeviceMatrix, down: DeviceMatrix, pipelines, x, y, ws: Workspace,
+              stream=None):
+    _check(lib().uw_mlp_block(C.byref(gate.mat), C.byref(up.mat), C.byref(down.mat), _pipes(pipelines),
+                              _ptr(x), x.shape[0], _ptr(y), ws.ptr, ws.nbytes, _stream(stream)), "uw_mlp_block")
+
+
+def autotune(dm: DeviceMatrix, batches, reps: int, x, y, ws: Workspace, flush=None, stream=None):
+    """Returns (choice[n_batches], us[n_batches, 4])."""
+    n = len(batches)
+    b = (C.c_int32 * n)(*batches)
+    choice = (C.c_int32 * n)()
+    us = (C.c_float * (4 * n))()
+    _check(lib().uw_autotune(C.byref(dm.mat), b, n, reps, _ptr(x), _ptr(y), _ptr(flush),
+                             0 if flush is None else flush.numel() * flush.element_size(), ws.ptr, ws.nbytes,
+                             choice, us, _stream(stream)), "uw_autotune")
+    return list(choice), np.array(list(us), dtype=np.float64).reshape(n, 4)
+
+
+def launch_count() -> int:
+    return int(lib().uw_launch_count())
+
+
+def version() -> int:
+    return int(lib().uw_version())

@@ -1,0 +1,62 @@
+"""Helpers for the GPU tests: upload seeded inputs, call the library through
+its C ABI, bring results back as BF16 bit patterns."""
+import numpy as np
+
+from mlp_huffman_coded_b200 import uw
+from oracle import uw_oracle as O
+
+TOL = 2e-2  # max |y - y_ref| <= TOL * rms(y_ref)
+
+
+def to_dev(a: np.ndarray):
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).cuda()
+    if a.dtype == np.uint32:
+        return torch.from_numpy(a.view(np.int32)).cuda()
+    return torch.from_numpy(a).cuda()
+
+
+def to_host_u16(t) -> np.ndarray:
+    return t.cpu().numpy().view(np.uint16)
+
+
+def empty_bf16(*shape):
+    import torch
+    return torch.empty(*shape, dtype=torch.int16, device="cuda")
+
+
+def bf16_f64(a: np.ndarray) -> np.ndarray:
+    return O.bf16_to_f64(a)
+
+
+def within_tol(y_u16: np.ndarray, y_ref: np.ndarray, tol: float = TOL):
+    y = bf16_f64(y_u16)
+    rms = float(np.sqrt(np.mean(y_ref ** 2)))
+    err = float(np.max(np.abs(y - y_ref)))
+    return err <= tol * rms, err, rms
+
+
+def device_matrix(w: np.ndarray, chunk_groups: int = 4, direct: bool = True):
+    enc = uw.encode(w, chunk_groups=chunk_groups)
+    dm = uw.DeviceMatrix(enc)
+    if direct:
+        ws = uw.Workspace(256)
+        dm.prepare_direct_palette(ws)
+        ws.check("transcode")
+    return dm
+
+
+def gemm_all(dm, x_dev, pipelines=(0, 1, 2, 3)):
+    """y for every pipeline (dict pipeline -> uint16 [B, rows])."""
+    B = x_dev.shape[0]
+    out = {}
+    nb = max(uw.workspace_bytes(dm, p, B) for p in pipelines)
+    ws = uw.Workspace(nb)
+    for p in pipelines:
+        y = empty_bf16(B, dm.rows)
+        uw.gemm(dm, p, x_dev, y, ws)
+        ws.check(f"gemm pipeline {p}")
+        out[p] = to_host_u16(y)
+    return out

@@ -1,0 +1,129 @@
+"""GPU parity of the three Huffman decoders (full BF16, exponent bytes,
+4-bit palette transcode) against the oracle: bit-exact, called through the
+C ABI."""
+import numpy as np
+import pytest
+
+from mlp_huffman_coded_b200 import synth
+from mlp_huffman_coded_b200 import uw
+from oracle import uw_oracle as O
+
+from gpu_util import device_matrix, to_dev, to_host_u16, empty_bf16
+
+pytestmark = pytest.mark.gpu
+
+
+def _decode_all(dm):
+    import torch
+    n = dm.rows * dm.cols
+    ws = uw.Workspace(256)
+    full = empty_bf16(n)
+    exp8 = torch.empty(n, dtype=torch.uint8, device="cuda")
+    idx4 = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
+    uw.decode_full(dm, full, ws)
+    uw.decode_exponent_only(dm, exp8, ws)
+    uw.transcode_palette(dm, idx4, ws)
+    ws.check("decode")
+    return (to_host_u16(full).reshape(dm.rows, dm.cols), exp8.cpu().numpy().reshape(dm.rows, dm.cols),
+            idx4.cpu().numpy().reshape(dm.rows, dm.cols // 2))
+
+
+def _expected_idx4(w, palette):
+    """Plain definition: palette index per element, 0 in verbatim groups."""
+    vg = np.repeat(O.verbatim_groups(w, palette), 64, axis=1)
+    idx = np.where(vg, 0, O.palette_lookup(palette)[(w >> 7) & 0xFF]).astype(np.uint8)
+    return (idx[:, 0::2] | (idx[:, 1::2] << 4)).astype(np.uint8)
+
+
+def _check(w, chunk_groups=4, oracle_stream=False):
+    if oracle_stream:
+        # decode the oracle's own encoding (no product code on the input side)
+        ref = O.encode(w, chunk_groups=chunk_groups)
+        enc = uw.encode(w, chunk_groups=chunk_groups)
+        enc.sm[:] = ref.sm.ravel()
+        enc.stream[:] = ref.stream
+        enc.chunk_bit_off[:] = ref.chunk_bit_off
+        enc.vflags[:] = ref.vflags.ravel()
+        enc.vprefix[:] = ref.vprefix
+        enc.verbatim[:] = ref.verbatim.ravel()
+        dm = uw.DeviceMatrix(enc)
+    else:
+        dm = device_matrix(w, chunk_groups, direct=False)
+    full, exp8, idx4 = _decode_all(dm)
+    assert np.array_equal(full, w)
+    assert np.array_equal(exp8, ((w >> 7) & 0xFF).astype(np.uint8))
+    assert np.array_equal(idx4, _expected_idx4(w, np.array(list(dm.enc.cb.palette), np.uint8)))
+
+
+def test_small_config_bit_exact():
+    p = synth.WORKLOADS["small_256x512"]
+    w = synth.weight_matrix(p["rows"], p["cols"], p["sigma"], p["outlier_rate"], p["outlier_scale"], p["seed"])
+    _check(w)
+    _check(w, oracle_stream=True)
+
+
+def test_every_bf16_pattern_bit_exact():
+    _check(synth.all_patterns_matrix(), chunk_groups=3)
+
+
+def test_special_values_and_degenerate_codes():
+    rng = np.random.default_rng(3)
+    exp = np.where(rng.random((8, 128)) < 0.7, 0, 255).astype(np.uint16)
+    w = ((rng.integers(0, 2, (8, 128)).astype(np.uint16) << 15) | (exp << 7)
+         | rng.integers(0, 128, (8, 128)).astype(np.uint16)).astype(np.uint16)
+    _check(w)
+    _check(np.full((3, 128), 120 << 7, dtype=np.uint16))          # one symbol
+    w = np.zeros((17, 64), dtype=np.uint16)                          # every group verbatim
+    for r in range(17):
+        w[r, :] = (10 + r) << 7
+        w[r, 7] = (100 + r) << 7
+    _check(w)
+
+
+@pytest.mark.parametrize("chunk_groups", [1, 2, 4, 5, 16])
+def test_chunk_sizes_and_ragged_tail(chunk_groups):
+    # 37 x 640: 370 groups, last chunk partial for most chunk sizes
+    _check(synth.weight_matrix(37, 640, 0.03, 2e-3, 300.0, 11), chunk_groups)
+
+
+def test_long_codes_use_the_slow_path():
+    # a very skewed exponent distribution: codes longer than 11 bits
+    rng = np.random.default_rng(9)
+    probs = 0.5 ** np.arange(1, 17)
+    probs /= probs.sum()
+    exp = rng.choice(np.arange(100, 116), size=(64, 1024), p=probs).astype(np.uint16)
+    w = ((exp << 7) | rng.integers(0, 128, exp.shape).astype(np.uint16)).astype(np.uint16)
+    enc = uw.encode(w)
+    assert enc.cb.max_len > 11
+    _check(w)
+
+
+def test_full_size_gate_matrix_bit_exact():
+    p = synth.WORKLOADS["gate_14336x4096"]
+    w = synth.weight_matrix(p["rows"], p["cols"], p["sigma"], p["outlier_rate"], p["outlier_scale"], p["seed"])
+    _check(w)
+
+
+def test_corrupt_offsets_are_reported_not_faulted():
+    w = synth.weight_matrix(64, 512, 0.02, 1e-3, 100.0, 5)
+    enc = uw.encode(w)
+    enc.chunk_bit_off[5] += 3           # chunk 4 ends early, chunk 5 starts late
+    dm = uw.DeviceMatrix(enc)
+    ws = uw.Workspace(256)
+    out = empty_bf16(64 * 512)
+    uw.decode_full(dm, out, ws)
+    assert ws.status() == uw.UW_ERR_CORRUPT
+    assert ws.status() == uw.UW_OK      # reading clears the sticky word
+
+
+def test_garbage_stream_stays_in_bounds():
+    w = synth.weight_matrix(64, 512, 0.02, 1e-3, 100.0, 6)
+    enc = uw.encode(w)
+    rng = np.random.default_rng(0)
+    enc.stream[:-2] = rng.integers(0, 2**32, enc.stream.size - 2, dtype=np.uint64).astype(np.uint32)
+    dm = uw.DeviceMatrix(enc)
+    ws = uw.Workspace(256)
+    import torch
+    out = torch.empty(64 * 512, dtype=torch.uint8, device="cuda")
+    uw.decode_exponent_only(dm, out, ws)
+    assert ws.status() == uw.UW_ERR_CORRUPT
