@@ -374,6 +374,57 @@ def run_gpu(args, world, rank, local):
     return 0
 
 
+def run_gemm_case(args, local):
+    """One matrix (gate, 14336x4096) through one pipeline: the unit the ncu
+    profiles in profiles/ are taken on.  Prints a small JSON line."""
+    import torch
+    from mlp_huffman_coded_b200 import synth, uw
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.mlp_block(D_MODEL, FFN, SIGMA, OUTLIER_RATE, OUTLIER_SCALE, SEED)[0]
+    enc = uw.encode(w)
+    dm = uw.DeviceMatrix(enc, device=dev)
+    ws = uw.Workspace(max(uw.workspace_bytes(dm, p, args.batch) for p in range(4)), device=dev)
+    dm.prepare_direct_palette(ws)
+    x = torch.from_numpy(synth.activations(args.batch, D_MODEL, 3).view(np.int16)).to(dev)
+    y = torch.empty(args.batch, FFN, dtype=torch.int16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    if args.pipeline == "bf16":
+        wd = torch.from_numpy(w.view(np.int16)).to(dev)
+        ws = uw.Workspace(uw.workspace_bytes(dm, uw.PIPE_BF16, args.batch), device=dev)
+
+        def call():
+            uw.gemm_bf16(wd, x, y, ws)
+    else:
+        pipe = uw.PIPELINES[args.pipeline]
+
+        def call():
+            uw.gemm(dm, pipe, x, y, ws)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    times = []
+    flush.fill_(1)
+    for _ in range(args.steps):
+        if not args.no_flush:
+            # read (not write) a buffer larger than L2, so L2 holds clean
+            # lines and the timed call pays no write-backs
+            flush.view(torch.int32).max()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    ws.check("gemm case")
+    t = float(np.median(times))
+    nbytes = dm.direct_palette_bytes() if args.pipeline == "direct" else None
+    print(json.dumps({"case": "gemm", "pipeline": args.pipeline, "batch": args.batch, "median_us": t,
+                      "min_us": float(np.min(times)), "direct_bytes": nbytes,
+                      "gbs": (nbytes / t / 1e3) if nbytes else None}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -383,11 +434,17 @@ def main(argv=None):
     ap.add_argument("--impl", default="uw", choices=["uw", "reference"])
     ap.add_argument("--ref-fraction", type=float, default=1 / 16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default="block", choices=["block", "gemm"],
+                    help="gemm: one 14336x4096 matrix through --pipeline (profiling unit)")
+    ap.add_argument("--pipeline", default="direct", choices=["full", "exponent", "transcode", "direct", "bf16"])
+    ap.add_argument("--no-flush", action="store_true", help="gemm case: leave L2 warm between calls")
     args = ap.parse_args(argv)
     world, rank, local = dist_init()
     try:
         if args.impl == "reference":
             return run_reference(args, world, rank)
+        if args.case == "gemm":
+            return run_gemm_case(args, local)
         return run_gpu(args, world, rank, local)
     finally:
         if world > 1:

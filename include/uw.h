@@ -48,6 +48,26 @@
  *               palette index per element, element 2j in the low nibble of
  *               byte j of the row, 2j+1 in the high nibble; 0 in verbatim
  *               groups.
+ *   pack        (optional, the direct-palette form built at load time by
+ *               uw_pack_direct_palette) one contiguous record per tile of
+ *               128 rows x 64 columns, tiles in (row block, column block)
+ *               order, record t starting at byte 16*pack_off[t]:
+ *                 [0, 8192)      sm bytes of the tile: row r, 16-byte chunk
+ *                                j at r*64 + 16*(j ^ ((r>>1)&3))
+ *                 [8192, 12288)  idx4 bytes of the tile: row r, chunk j at
+ *                                8192 + r*32 + 16*(j ^ ((r>>2)&1))
+ *                 [12288, 12304) 128-bit verbatim mask, bit r = row r's
+ *                                64-element group is verbatim
+ *                 [12304, 12416) zero (keeps every record 128-byte aligned)
+ *                 [12416, ...)   the first min(n, 32) verbatim rows of the
+ *                                tile (64 BF16 words each), in row order
+ *               Rows past `rows` are zero.  A tile with more than 32 verbatim
+ *               rows keeps the rest in the verbatim store only.  The chunk
+ *               order inside each 64-/32-byte row is the one that makes the
+ *               GEMM's row-per-thread 16-byte shared-memory reads free of
+ *               bank conflicts.
+ *   pack_off    uint32[n_tiles+1]: record offsets in 16-byte units
+ *               (uw_direct_pack_offsets), n_tiles = ceil(rows/128)*cols/64.
  *
  * Conventions for every call:
  *   - Every call returns a uw_status; nothing throws across the ABI.
@@ -143,6 +163,8 @@ typedef struct {
   const uint32_t* vprefix;
   const uint16_t* verbatim;  /* may be NULL when n_verbatim == 0 */
   const uint8_t* idx4;       /* may be NULL */
+  const uint8_t* pack;       /* direct-palette records, may be NULL */
+  const uint32_t* pack_off;  /* [n_tiles+1], NULL when pack is NULL */
 } uw_matrix;
 
 /* ---------------------------------------------------------------------------
@@ -175,6 +197,14 @@ UW_API uw_status uw_encode(const uint16_t* w_host, int64_t rows, int64_t cols, c
                     int32_t chunk_groups, uw_layout* io_layout, uint8_t* sm, uint32_t* stream,
                     uint32_t* chunk_bit_off, uint32_t* vflags, uint32_t* vprefix,
                     uint16_t* verbatim);
+
+/* Record offsets (16-byte units) of the direct-palette pack of a matrix,
+ * computed from its HOST vflags: pack_off[t+1] - pack_off[t] =
+ * (12416 + 128*min(verbatim rows of tile t, 32)) / 16.  pack_off_host holds
+ * n_tiles+1 entries; *pack_bytes (may be NULL) receives the total size.
+ * Errors: UW_ERR_INVALID_ARG, UW_ERR_UNSUPPORTED_SHAPE (pack above 64 GiB). */
+UW_API uw_status uw_direct_pack_offsets(const uw_layout* L, const uint32_t* vflags_host,
+                                        uint32_t* pack_off_host, uint64_t* pack_bytes);
 
 /* Host-side consistency check of a compressed matrix whose pointers are
  * HOST copies: canonical codebook with Kraft sum <= 1, offsets monotone and
@@ -229,15 +259,24 @@ UW_API uw_status uw_decode_exponent_only(const uw_matrix* m, uint8_t* out_exp8, 
 UW_API uw_status uw_transcode_palette(const uw_matrix* m, uint8_t* out_idx4, void* workspace,
                                size_t workspace_bytes, void* stream);
 
+/* Load-time assembly of the direct-palette pack (layout above) from sm,
+ * m->idx4 (must be set) and the verbatim store, so that the direct-palette
+ * GEMM streams one contiguous record per tile.  pack_off: device copy of the
+ * offsets from uw_direct_pack_offsets; out_pack: device buffer of
+ * 16*pack_off[n_tiles] bytes. */
+UW_API uw_status uw_pack_direct_palette(const uw_matrix* m, const uint32_t* pack_off,
+                                        uint8_t* out_pack, void* stream);
+
 /* ---------------------------------------------------------------------------
  * Reconstructive GEMM (section "How the reconstructive matmul works")
  * ------------------------------------------------------------------------- */
 
 /* y = x W^T with the direct-palette matrix: x is device BF16 [batch, cols]
  * row-major, y is device BF16 [batch, rows] row-major.  W is rebuilt tile by
- * tile on chip from sm + idx4 (+ verbatim rows, chosen once per 64-element
- * row) and fed to tcgen05 MMA with FP32 accumulation in tensor memory; y is
- * rounded to nearest-even BF16.  m->idx4 must be set.  The split of the K
+ * tile on chip from the pack records (sm + 4-bit indices + verbatim rows,
+ * chosen once per 64-element row) and fed to tcgen05 MMA with FP32
+ * accumulation in tensor memory; y is rounded to nearest-even BF16.
+ * m->pack and m->pack_off must be set (uw_pack_direct_palette).  The split of the K
  * loop across CTAs and the order of its reduction depend only on (rows, cols,
  * batch, SM count), so all pipelines give bit-identical y.
  * batch: 1..512.  Errors: UW_ERR_INVALID_ARG, UW_ERR_UNSUPPORTED_SHAPE,
@@ -294,7 +333,7 @@ UW_API uw_status uw_mlp_block(const uw_matrix* gate, const uw_matrix* up, const 
  * For each batch b in batches[0..n_batches): warm up, then run reps timed
  * calls (CUDA events on `stream`, preprocessing included), and keep the
  * median.  out_us[i*4 + p] = median microseconds of pipeline p at batches[i]
- * (+INF when the pipeline is unavailable, e.g. DIRECT without m->idx4);
+ * (+INF when the pipeline is unavailable, e.g. DIRECT without m->pack);
  * out_choice[i] = the pipeline with the smallest time.  x/y: device buffers
  * of at least max(batches)*cols / max(batches)*rows BF16 values used as
  * inputs/outputs of the timed calls.  flush/flush_bytes (optional, may be

@@ -35,7 +35,7 @@ extern "C" uw_status uw_autotune(const uw_matrix* m, const int32_t* batches, int
     for (int p = UW_PIPE_FULL; p <= UW_PIPE_DIRECT && st == UW_OK; ++p) {
       float& slot = out_us[bi * 4 + p];
       slot = INFINITY;
-      if (p == UW_PIPE_DIRECT && !m->idx4) continue;
+      if (p == UW_PIPE_DIRECT && (!m->pack || !m->pack_off)) continue;
       if (uw_workspace_bytes(&m->L, p, B) > ws_bytes) continue;
       // warm-up (also surfaces argument errors)
       for (int w = 0; w < 2 && st == UW_OK; ++w) st = uw_gemm(m, p, x, B, y, ws, ws_bytes, s);

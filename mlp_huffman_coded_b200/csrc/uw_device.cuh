@@ -221,15 +221,24 @@ struct PaletteTables {
   uint32_t keep;                    // 0x7F7F7F7F or 0xFFFFFFFF (uniform case)
 };
 
+// PTX prmt in its default mode, where bit 3 of each selector nibble asks for
+// the selected byte's top bit to be replicated.  (The __byte_perm intrinsic
+// is defined on 3-bit selectors only, so it cannot be used for this.)
+__device__ __forceinline__ uint32_t prmt_sx(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
 __device__ __forceinline__ uint32_t lookup4_uniform(const PaletteTables& p, uint32_t nib) {
-  const uint32_t a = __byte_perm(p.lo0, p.lo1, nib);
-  const uint32_t b = __byte_perm(p.hi0, p.hi1, nib ^ 0x8888u);
+  const uint32_t a = prmt_sx(p.lo0, p.lo1, nib);
+  const uint32_t b = prmt_sx(p.hi0, p.hi1, nib ^ 0x8888u);
   return a & b & p.keep;
 }
 
 __device__ __forceinline__ uint32_t lookup4_mixed(const PaletteTables& p, uint32_t nib) {
-  const uint32_t a = __byte_perm(p.lo0, p.lo1, nib) & __byte_perm(p.hi0, p.hi1, nib ^ 0x8888u);
-  const uint32_t b = __byte_perm(p.b7lo0, p.b7lo1, nib) & __byte_perm(p.b7hi0, p.b7hi1, nib ^ 0x8888u);
+  const uint32_t a = prmt_sx(p.lo0, p.lo1, nib) & prmt_sx(p.hi0, p.hi1, nib ^ 0x8888u);
+  const uint32_t b = prmt_sx(p.b7lo0, p.b7lo1, nib) & prmt_sx(p.b7hi0, p.b7hi1, nib ^ 0x8888u);
   return a & ((b << 1) | 0x7F7F7F7Fu);
 }
 

@@ -30,6 +30,7 @@
 //  * Every barrier wait is bounded in time; a timeout records UW_ERR_TIMEOUT,
 //    drains in-flight copies and frees tensor memory before returning.
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -40,11 +41,15 @@ namespace uw {
 
 namespace {
 
-constexpr int kThreads = 320;  // 10 warps
+// Warp roles: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), then
+// `groups` rebuild warpgroups of 4 warps (group g rebuilds the stages of
+// units i with i % groups == g, so several stages are rebuilt at once), then
+// 4 epilogue warps.
+constexpr int kMaxGroups = 2;
+constexpr int kMaxThreads = 32 * (6 + 4 * kMaxGroups);
 constexpr int kWarpProducer = 0;
 constexpr int kWarpMma = 1;
-constexpr int kWarpRebuild0 = 2;  // warps 2..5
-constexpr int kWarpEpi0 = 6;      // warps 6..9
+constexpr int kWarpRebuild0 = 2;
 constexpr int kVCap = 16;         // verbatim rows staged on chip per tile
 constexpr int kMaxStages = 8;
 constexpr uint32_t kTmemCols = 512;
@@ -53,7 +58,16 @@ constexpr uint32_t kAStageCol0 = 256;
 constexpr size_t kSmemLimit = 227 * 1024;
 constexpr size_t kSmemFloor = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
 
-enum KernelLoader { kBF16 = 0, kEXP8 = 1, kIDX4U = 2, kIDX4M = 3 };
+// Tile loaders: BF16 tiles (full-decode pipeline and the uncompressed
+// comparator), sm + exponent bytes (exponent-only pipeline), row-major sm +
+// 4-bit indices + verbatim store (run-time transcode pipeline) and the
+// direct-palette pack records; U/M = palette lookup for a uniform / mixed
+// top exponent bit.
+enum KernelLoader { kBF16 = 0, kEXP8 = 1, kIDX4U = 2, kIDX4M = 3, kPACKU = 4, kPACKM = 5 };
+__host__ __device__ constexpr bool loader_pack(int L) { return L == kPACKU || L == kPACKM; }
+__host__ __device__ constexpr bool loader_uniform(int L) { return L == kIDX4U || L == kPACKU; }
+constexpr uint32_t kRecIdx = 8192, kRecMask = 12288, kRecVerb = 12416, kRecVCap = 32;
+constexpr uint32_t kRecMax = kRecVerb + kRecVCap * 128;
 
 struct KParams {
   int N, K, B, KB, n_ntiles, ntile;
@@ -75,13 +89,21 @@ struct KParams {
   uint32_t* status;
   PaletteTables pal;
   uint32_t idesc;
+  int groups;  // rebuild warpgroups
+  int vcap;    // verbatim rows staged on chip per tile
+  int n_acc;   // accumulator buffers in TMEM (2 alternate segments when they fit)
+  const uint8_t* pack;
+  const uint32_t* pack_off;
+  uint32_t off_rec;   // pack record inside a stage
+  uint32_t soff_off;  // shared-memory copy of this CTA's record offsets
+  int n_soff;         // its capacity in words
 };
 
 struct Bars {
   uint64_t full[kMaxStages];
   uint64_t rebuilt[kMaxStages];
   uint64_t empty[kMaxStages];
-  uint64_t acc_full, acc_empty, drain;
+  uint64_t acc_full[2], acc_empty[2], drain;
   uint64_t meta_full[2];
   uint32_t tmem_base;
   uint32_t abort;
@@ -116,6 +138,15 @@ __device__ __forceinline__ bool group_and(bool v) {  // warps 6..9 (named barrie
 __device__ __forceinline__ void group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+
+// y[b, n] = bf16(v), or bf16(SiLU(gate[b, n]) * bf16(v)) for the fused
+// SwiGLU epilogue.
+__device__ __forceinline__ void store_out(const KParams& p, int b, int64_t n, float v) {
+  __nv_bfloat16 val = __float2bfloat16_rn(v);
+  const int64_t i = static_cast<int64_t>(b) * p.N + n;
+  if (p.gate) val = swiglu_bf16(reinterpret_cast<const __nv_bfloat16*>(p.gate)[i], val);
+  reinterpret_cast<__nv_bfloat16*>(p.y)[i] = val;
+}
 
 // ----------------------------- tile rebuild ---------------------------------
 // Each rebuild thread owns one row r of the 128-row tile and produces the 64
@@ -168,7 +199,7 @@ __device__ __forceinline__ void rebuild_row(const uint8_t* stage, const KParams&
       for (int h = 0; h < 2; ++h) {
         const uint32_t nib = iw[2 * j + h];  // 8 indices: elements 16j + 8h .. +7
         uint32_t e0, e1;
-        if constexpr (L == kIDX4U) {
+        if constexpr (loader_uniform(L)) {
           e0 = lookup4_uniform(p.pal, nib);
           e1 = lookup4_uniform(p.pal, nib >> 16);
         } else {
@@ -184,10 +215,11 @@ __device__ __forceinline__ void rebuild_row(const uint8_t* stage, const KParams&
 
 // ------------------------------- the kernel ----------------------------------
 template <int L>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kMaxThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wa,
                 const __grid_constant__ CUtensorMap tm_wb, const KParams p) {
-  constexpr bool kIdx4 = (L == kIDX4U || L == kIDX4M);
+  constexpr bool kIdx4 = (L == kIDX4U || L == kIDX4M);  // row-major indices + verbatim store
+  constexpr bool kPack = loader_pack(L);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Bars* bars = reinterpret_cast<Bars*>(smem + p.bar_off);
@@ -196,6 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int64_t u0 = unit_begin(blockIdx.x, p);
   const int64_t u1 = unit_begin(blockIdx.x + 1, p);
   const int S = p.stages;
+  const int G = p.groups;
+  const int warp_epi0 = kWarpRebuild0 + 4 * G;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -203,8 +237,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars->rebuilt[s], 4);
       mbar_init(&bars->empty[s], 1);
     }
-    mbar_init(&bars->acc_full, 1);
-    mbar_init(&bars->acc_empty, 4);
+    mbar_init(&bars->acc_full[0], 1);
+    mbar_init(&bars->acc_full[1], 1);
+    mbar_init(&bars->acc_empty[0], 4);
+    mbar_init(&bars->acc_empty[1], 4);
     mbar_init(&bars->drain, 1);
     mbar_init(&bars->meta_full[0], 1);
     mbar_init(&bars->meta_full[1], 1);
@@ -218,8 +254,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == kWarpProducer && lane == 0) {
     prefetch_tensormap(&tm_x);
-    prefetch_tensormap(&tm_wa);
-    if (L != kBF16) prefetch_tensormap(&tm_wb);
+    if (!kPack) prefetch_tensormap(&tm_wa);
+    if (L != kBF16 && !kPack) prefetch_tensormap(&tm_wb);
   }
   tc_fence_before();
   __syncthreads();
@@ -259,18 +295,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       issue_meta(mt_first, 0);
       if (mt_first + 1 <= mt_last) issue_meta(mt_first + 1, 1);
     }
+    // pack records: offsets of every record this CTA can touch
+    uint32_t* soff = reinterpret_cast<uint32_t*>(smem + p.soff_off);
+    const int64_t pt_min = static_cast<int64_t>(mt_first) * p.KB;
+    if (kPack) {
+      const int64_t n_tiles_total = static_cast<int64_t>((p.N + 127) / 128) * p.KB;
+      const int64_t want = static_cast<int64_t>(mt_last - mt_first + 1) * p.KB + 1;
+      const int64_t cnt = want < p.n_soff ? want : p.n_soff;
+      for (int64_t w = lane; w < cnt; w += 32)
+        soff[w] = (pt_min + w <= n_tiles_total) ? __ldg(p.pack_off + pt_min + w) : 0u;
+      __syncwarp();
+    }
     int cur_mt = -1;
     int64_t i = 0;
+    // the loop advances (stage, use) and (row block, batch tile, k-block)
+    // incrementally: no division per unit
+    int s = 0;
+    uint32_t k = 0;
+    int kb, mt, nt;
+    {
+      const int64_t t0 = u0 / p.KB;
+      kb = static_cast<int>(u0 - t0 * p.KB);
+      mt = static_cast<int>(t0 / p.n_ntiles);
+      nt = static_cast<int>(t0 - static_cast<int64_t>(mt) * p.n_ntiles);
+    }
     for (int64_t u = u0; u < u1; ++u, ++i) {
-      const int s = static_cast<int>(i % S);
-      const uint32_t k = static_cast<uint32_t>(i / S);
+      if (i > 0) {
+        if (++s == S) {
+          s = 0;
+          ++k;
+        }
+        if (++kb == p.KB) {
+          kb = 0;
+          if (++nt == p.n_ntiles) {
+            nt = 0;
+            ++mt;
+          }
+        }
+      }
       if (k > 0 && !warp_wait(&bars->empty[s], (k - 1) & 1, bars, p.status)) break;
-      const int64_t t = u / p.KB;
-      const int kb = static_cast<int>(u - t * p.KB);
-      const int mt = static_cast<int>(t / p.n_ntiles);
-      const int nt = static_cast<int>(t - static_cast<int64_t>(mt) * p.n_ntiles);
       uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
       uint32_t tx = p.x_bytes + p.wa_bytes + p.wb_bytes;
+      uint32_t rec_o0 = 0, rec_bytes = 0;
+      if (kPack) {
+        const int64_t slot = static_cast<int64_t>(mt) * p.KB + kb - pt_min;
+        if (slot + 1 < p.n_soff) {
+          rec_o0 = soff[slot];
+          rec_bytes = (soff[slot + 1] - rec_o0) * 16u;
+        }
+        if (rec_bytes < kRecVerb || rec_bytes > kRecMax || ((rec_bytes - kRecVerb) & 127)) {
+          // inconsistent offsets: load nothing for this tile (bounded garbage)
+          if (lane == 0) record_status(p.status, UW_ERR_CORRUPT);
+          rec_bytes = 0;
+        }
+        tx = p.x_bytes + rec_bytes;
+      }
       int vq_dst[4];
       int64_t vq_src[4];
       if (kIdx4) {
@@ -304,7 +383,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) {
         mbar_arrive_expect_tx(&bars->full[s], tx);
         tma_load_2d(stage + p.off_x, &tm_x, kb * 64, nt * p.ntile, &bars->full[s]);
-        if (L == kIDX4U || L == kIDX4M) {
+        if (kPack) {
+          if (rec_bytes)
+            bulk_load(stage + p.off_rec, p.pack + static_cast<uint64_t>(rec_o0) * 16, rec_bytes, &bars->full[s]);
+        } else if (L == kIDX4U || L == kIDX4M) {
           tma_load_2d(stage + p.off_wa, &tm_wa, kb * 64, mt * 128, &bars->full[s]);
           tma_load_2d(stage + p.off_wb, &tm_wb, kb * 32, mt * 128, &bars->full[s]);
         } else if (L == kEXP8) {
@@ -333,53 +415,81 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == kWarpMma) {
     // ----------------------------- MMA issuer -------------------------------
+    // One thread issues every MMA.  An M=128, K=16 tcgen05.mma occupies the
+    // tensor pipe for a fixed ~100+ cycles even at N=16, so at decode-sized
+    // batches this thread sets the pace: its loop carries all indices
+    // incrementally and does nothing but wait, issue and commit.
     if (lane == 0) {
-      uint32_t seg = 0;
-      int64_t i = 0;
-      for (int64_t u = u0; u < u1; ++u, ++i) {
-        const int s = static_cast<int>(i % S);
-        const uint32_t k = static_cast<uint32_t>(i / S);
-        const int kb = static_cast<int>(u % p.KB);
-        const bool first = (u == u0) || kb == 0;
+      int s = 0;
+      uint32_t k = 0;
+      int kb = static_cast<int>(u0 % p.KB);
+      uint32_t ab = 0;                    // accumulator buffer of this segment
+      uint32_t use_par[2] = {0u, 0u};     // completed-drain parity per buffer
+      uint32_t used[2] = {0u, 0u};        // segments already run per buffer
+      const uint32_t acc_stride = static_cast<uint32_t>(p.ntile);
+      const uint64_t b_desc0 = smem_desc_sw128(smem_u32(smem + p.off_x));
+      const uint64_t b_step = static_cast<uint64_t>(p.stage_bytes >> 4);
+      bool first = true;
+      for (int64_t u = u0; u < u1; ++u) {
         const bool last = (u == u1 - 1) || kb == p.KB - 1;
-        if (first && seg > 0) {
-          if (!mbar_wait(&bars->acc_empty, (seg - 1) & 1, &bars->abort, p.status)) break;
+        const uint32_t d_tmem = tmem + kAccCol + ab * acc_stride;
+        if (first && used[ab] > 0) {
+          if (!mbar_wait(&bars->acc_empty[ab], use_par[ab], &bars->abort, p.status)) break;
+          use_par[ab] ^= 1u;
           tc_fence_after();
         }
         if (!mbar_wait(&bars->full[s], k & 1, &bars->abort, p.status)) break;
         if (!mbar_wait(&bars->rebuilt[s], k & 1, &bars->abort, p.status)) break;
         tc_fence_after();
         const uint32_t a_tmem = tmem + kAStageCol0 + static_cast<uint32_t>(s) * 32;
-        const uint64_t b_desc = smem_desc_sw128(smem_u32(smem + static_cast<size_t>(s) * p.stage_bytes + p.off_x));
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          mma_ts(tmem + kAccCol, a_tmem + j * 8, b_desc + static_cast<uint64_t>(j * 2), p.idesc,
-                 (first && j == 0) ? 0u : 1u);
+        const uint64_t b_desc = b_desc0 + static_cast<uint64_t>(s) * b_step;
+        mma_ts(d_tmem, a_tmem + 0, b_desc + 0, p.idesc, first ? 0u : 1u);
+        mma_ts(d_tmem, a_tmem + 8, b_desc + 2, p.idesc, 1u);
+        mma_ts(d_tmem, a_tmem + 16, b_desc + 4, p.idesc, 1u);
+        mma_ts(d_tmem, a_tmem + 24, b_desc + 6, p.idesc, 1u);
         tc_commit(&bars->empty[s]);
         if (last) {
-          tc_commit(&bars->acc_full);
-          ++seg;
+          tc_commit(&bars->acc_full[ab]);
+          ++used[ab];
+          if (p.n_acc == 2) ab ^= 1u;
         }
+        first = last;
+        if (++s == S) {
+          s = 0;
+          ++k;
+        }
+        if (++kb == p.KB) kb = 0;
       }
       // every MMA issued so far must finish before tensor memory is freed
       tc_commit(&bars->drain);
       mbar_wait(&bars->drain, 0, nullptr, p.status);
     }
     __syncwarp();
-  } else if (warp < kWarpEpi0) {
+  } else if (warp < warp_epi0) {
     // ------------------------------- rebuild --------------------------------
     const int q = warp & 3;
     const int r = q * 32 + lane;
-    int64_t i = 0;
-    for (int64_t u = u0; u < u1; ++u, ++i) {
-      const int s = static_cast<int>(i % S);
-      const uint32_t k = static_cast<uint32_t>(i / S);
+    const int grp = (warp - kWarpRebuild0) >> 2;
+    int s = grp;  // group g takes units u0+g, u0+g+G, ... (G <= S)
+    uint32_t k = 0;
+    while (s >= S) {
+      s -= S;
+      ++k;
+    }
+    for (int64_t u = u0 + grp; u < u1; u += G) {
+      if (u != u0 + grp) {
+        s += G;
+        if (s >= S) {
+          s -= S;
+          ++k;
+        }
+      }
       if (!warp_wait(&bars->full[s], k & 1, bars, p.status)) break;
       tc_fence_after();
       const uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
       uint32_t o[32];
       rebuild_row<L>(stage, p, r, o);
-      if (kIdx4) {
+      if (kIdx4 || kPack) {
         // verbatim rows: one flag bit per row and k-block, no per-element test
         const uint32_t* hdr = reinterpret_cast<const uint32_t*>(stage + p.off_hdr);
         const uint32_t m = hdr[q];
@@ -387,7 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           int idx = __popc(m & ((1u << lane) - 1));
           for (int qq = 0; qq < q; ++qq) idx += __popc(hdr[qq]);
           const uint4* src;
-          if (idx < kVCap) {
+          if (idx < p.vcap) {
             src = reinterpret_cast<const uint4*>(stage + p.off_verb + idx * 128);
           } else {
             // more verbatim rows than staged slots: read this one from HBM
@@ -429,58 +539,90 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int64_t c_first = unit_owner(t * p.KB, p);
       const int64_t c_last = unit_owner(t * p.KB + p.KB - 1, p);
       const int ncontrib = static_cast<int>(c_last - c_first + 1);
-      bool ok = mbar_wait(&bars->acc_full, seg & 1, &bars->abort, p.status);
+      const uint32_t ab = seg % p.n_acc, use = seg / p.n_acc;
+      bool ok = mbar_wait(&bars->acc_full[ab], use & 1, &bars->abort, p.status);
       ok = __all_sync(0xFFFFFFFFu, ok);
       ok = group_and(ok);
       if (!ok) break;
       tc_fence_after();
       const int64_t n = static_cast<int64_t>(mt) * 128 + r;
       const bool row_ok = n < p.N;
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + kAccCol;
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + kAccCol + ab * static_cast<uint32_t>(p.ntile);
       const int64_t slot0 = t + c_first;
+      // partial sums: slot-major, then row, then column, so one thread owns a
+      // contiguous run of ntile floats and moves it with 16-byte accesses
+      float* my_part = p.partials + ((slot0 + (blockIdx.x - c_first)) * 128 + r) * p.ntile;
       for (int cc = 0; cc < p.ntile / 16; ++cc) {
         uint32_t v[16];
         tmem_ld16(taddr + cc * 16, v);
         tc_wait_ld();
+        if (ncontrib == 1) {
+          if (row_ok) {
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int col = cc * 16 + jj;
-          const int b = nt * p.ntile + col;
-          if (ncontrib == 1) {
-            if (row_ok && b < p.B) {
-              __nv_bfloat16 val = __float2bfloat16_rn(__uint_as_float(v[jj]));
-              if (p.gate) val = swiglu_bf16(reinterpret_cast<const __nv_bfloat16*>(p.gate)[static_cast<int64_t>(b) * p.N + n], val);
-              reinterpret_cast<__nv_bfloat16*>(p.y)[static_cast<int64_t>(b) * p.N + n] = val;
+            for (int jj = 0; jj < 16; ++jj) {
+              const int b = nt * p.ntile + cc * 16 + jj;
+              if (b < p.B) store_out(p, b, n, __uint_as_float(v[jj]));
             }
-          } else {
-            const int64_t slot = slot0 + (blockIdx.x - c_first);
-            p.partials[(slot * p.ntile + col) * 128 + r] = __uint_as_float(v[jj]);
           }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(my_part + cc * 16);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4)
+            dst[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
+                                  __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->acc_empty);
+      if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);
       if (ncontrib > 1) {
         __threadfence();
         group_sync();
-        if (warp == kWarpEpi0 && lane == 0) {
+        if (warp == warp_epi0 && lane == 0) {
           const uint32_t old = atomicAdd(p.counters + t, 1u);
           bars->is_last = (old == static_cast<uint32_t>(ncontrib - 1)) ? 1u : 0u;
         }
         group_sync();
         if (bars->is_last) {
           __threadfence();
-          for (int col = 0; col < p.ntile; ++col) {
-            const int b = nt * p.ntile + col;
-            if (!row_ok || b >= p.B) continue;
-            float acc = 0.0f;
-            for (int jc = 0; jc < ncontrib; ++jc) acc += __ldcg(p.partials + ((slot0 + jc) * p.ntile + col) * 128 + r);
-            __nv_bfloat16 val = __float2bfloat16_rn(acc);
-            if (p.gate) val = swiglu_bf16(reinterpret_cast<const __nv_bfloat16*>(p.gate)[static_cast<int64_t>(b) * p.N + n], val);
-            reinterpret_cast<__nv_bfloat16*>(p.y)[static_cast<int64_t>(b) * p.N + n] = val;
+          // fixed order: contributor 0, 1, ... (the CTA order), independent of
+          // which CTA finished last; 16 columns at a time, all loads of a
+          // chunk issued before any is summed
+          for (int cc = 0; cc < p.ntile / 16; ++cc) {
+            float acc[16];
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) acc[jj] = 0.0f;
+            for (int jc = 0; jc < ncontrib; jc += 4) {
+              float4 ld[4][4];
+#pragma unroll
+              for (int a = 0; a < 4; ++a)
+                if (jc + a < ncontrib) {
+                  const float4* src = reinterpret_cast<const float4*>(
+                      p.partials + ((slot0 + jc + a) * 128 + r) * p.ntile + cc * 16);
+#pragma unroll
+                  for (int q4 = 0; q4 < 4; ++q4) ld[a][q4] = __ldcg(src + q4);
+                }
+#pragma unroll
+              for (int a = 0; a < 4; ++a)
+                if (jc + a < ncontrib) {
+#pragma unroll
+                  for (int q4 = 0; q4 < 4; ++q4) {
+                    acc[4 * q4] += ld[a][q4].x;
+                    acc[4 * q4 + 1] += ld[a][q4].y;
+                    acc[4 * q4 + 2] += ld[a][q4].z;
+                    acc[4 * q4 + 3] += ld[a][q4].w;
+                  }
+                }
+            }
+            if (row_ok) {
+#pragma unroll
+              for (int jj = 0; jj < 16; ++jj) {
+                const int b = nt * p.ntile + cc * 16 + jj;
+                if (b < p.B) store_out(p, b, n, acc[jj]);
+              }
+            }
           }
-          if (warp == kWarpEpi0 && lane == 0) p.counters[t] = 0;
+          if (warp == warp_epi0 && lane == 0) p.counters[t] = 0;
         }
       }
       ++seg;
@@ -507,35 +649,81 @@ __global__ void swiglu_kernel(const __nv_bfloat16* __restrict__ g, const __nv_bf
 
 struct Layout {
   int stages = 0;
-  uint32_t stage_bytes = 0, off_x = 0, off_wa = 0, off_wb = 0, off_verb = 0, off_hdr = 0;
+  uint32_t stage_bytes = 0, off_x = 0, off_wa = 0, off_wb = 0, off_verb = 0, off_hdr = 0, off_rec = 0;
   uint32_t x_bytes = 0, wa_bytes = 0, wb_bytes = 0;
-  uint32_t meta_off = 0, meta_slot_words = 0, bar_off = 0;
+  uint32_t meta_off = 0, meta_slot_words = 0, bar_off = 0, soff_off = 0;
+  int n_soff = 0, vcap = 0;
   size_t smem = 0;
 };
 
 uint32_t a1024(uint32_t v) { return (v + 1023u) & ~1023u; }
 
-bool make_layout(int loader, int ntile, int wpr, Layout* out) {
+// Pipeline depth cap (UW_MAX_STAGES overrides, for tuning).
+int max_stages() {
+  static int v = [] {
+    const char* e = std::getenv("UW_MAX_STAGES");
+    int x = e ? std::atoi(e) : kMaxStages;
+    return x < 2 ? 2 : (x > kMaxStages ? kMaxStages : x);
+  }();
+  return v;
+}
+
+// Rebuild warpgroups per CTA (UW_REBUILD_GROUPS overrides, for tuning).
+int rebuild_groups() {
+  static int g = [] {
+    const char* e = std::getenv("UW_REBUILD_GROUPS");
+    int v = e ? std::atoi(e) : 2;
+    return v < 1 ? 1 : (v > kMaxGroups ? kMaxGroups : v);
+  }();
+  return g;
+}
+
+// Shared-memory plan of one launch.  Every tile region starts on a 1024-byte
+// boundary (the 128-byte swizzle of the activation tile repeats every 1024).
+bool make_layout(int loader, const GemmPlan& plan, int wpr, Layout* out) {
   Layout l;
-  l.x_bytes = static_cast<uint32_t>(ntile) * 128;
+  l.x_bytes = static_cast<uint32_t>(plan.ntile) * 128;
   const bool idx4 = loader == kIDX4U || loader == kIDX4M;
-  l.wa_bytes = loader == kBF16 ? 16384u : 8192u;
-  l.wb_bytes = loader == kBF16 ? 0u : (loader == kEXP8 ? 8192u : 4096u);
+  const bool pack = loader_pack(loader);
   l.off_x = 0;
-  l.off_wa = a1024(l.off_x + l.x_bytes);
-  l.off_wb = a1024(l.off_wa + l.wa_bytes);
-  l.off_verb = a1024(l.off_wb + l.wb_bytes);
-  l.off_hdr = l.off_verb + (idx4 ? kVCap * 128u : 0u);
-  l.stage_bytes = a1024(l.off_hdr + (idx4 ? 64u : 0u));
+  if (pack) {
+    l.off_rec = a1024(l.x_bytes);
+    l.off_wa = l.off_rec;
+    l.off_wb = l.off_rec + kRecIdx;
+    l.off_hdr = l.off_rec + kRecMask;
+    l.off_verb = l.off_rec + kRecVerb;
+    l.vcap = kRecVCap;
+    l.stage_bytes = a1024(l.off_rec + kRecMax);
+  } else {
+    l.wa_bytes = loader == kBF16 ? 16384u : 8192u;
+    l.wb_bytes = loader == kBF16 ? 0u : (loader == kEXP8 ? 8192u : 4096u);
+    l.off_wa = a1024(l.off_x + l.x_bytes);
+    l.off_wb = a1024(l.off_wa + l.wa_bytes);
+    l.off_verb = a1024(l.off_wb + l.wb_bytes);
+    l.off_hdr = l.off_verb + (idx4 ? kVCap * 128u : 0u);
+    l.vcap = kVCap;
+    l.stage_bytes = a1024(l.off_hdr + (idx4 ? 64u : 0u));
+  }
   l.meta_slot_words = idx4 ? 128u * static_cast<uint32_t>(wpr) : 0u;
   const uint32_t meta_bytes = a1024(2u * 2u * l.meta_slot_words * 4u);
-  const uint32_t fixed = meta_bytes + a1024(sizeof(Bars)) + 1024u;  // + alignment slack
+  // pack: record offsets of every tile one CTA can reach (its units span at
+  // most `span` row blocks)
+  if (pack) {
+    const int64_t per_cta = (plan.units + plan.grid - 1) / plan.grid;
+    const int64_t per_mt = static_cast<int64_t>(plan.KB) * plan.n_ntiles;
+    const int64_t span = (per_cta + per_mt - 1) / per_mt + 1;
+    l.n_soff = static_cast<int>(span * plan.KB + 1);
+  }
+  const uint32_t soff_bytes = a1024(static_cast<uint32_t>(l.n_soff) * 4u);
+  const uint32_t fixed = meta_bytes + soff_bytes + a1024(sizeof(Bars)) + 1024u;  // + alignment slack
+  if (fixed >= kSmemLimit) return false;
   int stages = static_cast<int>((kSmemLimit - fixed) / l.stage_bytes);
-  stages = std::min(stages, kMaxStages);
+  stages = std::min(stages, max_stages());
   if (stages < 2) return false;
   l.stages = stages;
   l.meta_off = static_cast<uint32_t>(stages) * l.stage_bytes;
-  l.bar_off = l.meta_off + meta_bytes;
+  l.soff_off = l.meta_off + meta_bytes;
+  l.bar_off = l.soff_off + soff_bytes;
   l.smem = std::max<size_t>(static_cast<size_t>(l.bar_off) + a1024(sizeof(Bars)) + 1024u, kSmemFloor);
   *out = l;
   return true;
@@ -553,7 +741,7 @@ uw_status launch_kernel(const CUtensorMap& x, const CUtensorMap& wa, const CUten
                                               static_cast<int>(kSmemLimit));
   });
   if (attr_err[dev & 63] != cudaSuccess) return UW_ERR_CUDA;
-  gemm_kernel<L><<<kp.grid, kThreads, smem, s>>>(x, wa, wb, kp);
+  gemm_kernel<L><<<kp.grid, 32 * (6 + 4 * kp.groups), smem, s>>>(x, wa, wb, kp);
   note_launch();
   return cuda_status(cudaGetLastError());
 }
@@ -601,6 +789,13 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   } else if (a.loader == kLoaderEXP8) {
     if (!a.sm || !a.aux || !aligned16(a.sm) || !aligned16(a.aux)) return UW_ERR_INVALID_ARG;
     kl = kEXP8;
+  } else if (a.loader == kLoaderPACK) {
+    if (!a.pack || !a.pack_off || !a.vflags || !a.vprefix || !a.palette) return UW_ERR_INVALID_ARG;
+    if (!aligned16(a.pack) || !aligned16(a.vflags) || !aligned16(a.vprefix) || (a.verbatim && !aligned16(a.verbatim)))
+      return UW_ERR_INVALID_ARG;
+    bool mixed = false;
+    pal = palette_tables(a.palette, a.code_len, &mixed);
+    kl = (mixed || a.force_mixed_palette) ? kPACKM : kPACKU;
   } else {
     if (!a.sm || !a.aux || !a.vflags || !a.vprefix || !a.palette) return UW_ERR_INVALID_ARG;
     if (!aligned16(a.sm) || !aligned16(a.aux) || !aligned16(a.vflags) || !aligned16(a.vprefix) ||
@@ -611,14 +806,17 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
     kl = (mixed || a.force_mixed_palette) ? kIDX4M : kIDX4U;
   }
   Layout lay;
-  if (!make_layout(kl, plan.ntile, a.wpr, &lay)) return UW_ERR_UNSUPPORTED_SHAPE;
+  if (!make_layout(kl, plan, a.wpr, &lay)) return UW_ERR_UNSUPPORTED_SHAPE;
 
   CUtensorMap tx, twa, twb;
   std::memset(&twb, 0, sizeof(twb));
   if ((st = make_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, a.K, a.B, a.K * 2, 64, plan.ntile,
                                CU_TENSOR_MAP_SWIZZLE_128B)) != UW_OK)
     return st;
-  if (kl == kBF16) {
+  if (loader_pack(kl)) {
+    twa = tx;  // unused: pack records arrive by bulk copy
+    twb = tx;
+  } else if (kl == kBF16) {
     if ((st = make_tensor_map_2d(&twa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.wbf16, a.K, a.N, a.K * 2, 64, 128,
                                  CU_TENSOR_MAP_SWIZZLE_128B)) != UW_OK)
       return st;
@@ -671,12 +869,22 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.partials = reinterpret_cast<float*>(ws + kWsHeader + plan.counter_bytes);
   kp.pal = pal;
   kp.idesc = idesc_bf16_f32(plan.ntile);
+  kp.groups = rebuild_groups();
+  kp.vcap = lay.vcap;
+  kp.n_acc = 2 * plan.ntile <= 256 ? 2 : 1;
+  kp.pack = a.pack;
+  kp.pack_off = a.pack_off;
+  kp.off_rec = lay.off_rec;
+  kp.soff_off = lay.soff_off;
+  kp.n_soff = lay.n_soff;
 
   switch (kl) {
     case kBF16: return launch_kernel<kBF16>(tx, twa, twb, kp, lay.smem, s);
     case kEXP8: return launch_kernel<kEXP8>(tx, twa, twb, kp, lay.smem, s);
     case kIDX4U: return launch_kernel<kIDX4U>(tx, twa, twb, kp, lay.smem, s);
-    default: return launch_kernel<kIDX4M>(tx, twa, twb, kp, lay.smem, s);
+    case kIDX4M: return launch_kernel<kIDX4M>(tx, twa, twb, kp, lay.smem, s);
+    case kPACKU: return launch_kernel<kPACKU>(tx, twa, twb, kp, lay.smem, s);
+    default: return launch_kernel<kPACKM>(tx, twa, twb, kp, lay.smem, s);
   }
 }
 
@@ -735,14 +943,20 @@ uw_status run_pipeline(const uw_matrix* m, int pipeline, const uint16_t* x, int3
       a.sm = m->sm;
       a.aux = static_cast<const uint8_t*>(scratch);
       break;
-    case UW_PIPE_TRANSCODE:
-    case UW_PIPE_DIRECT: {
-      const uint8_t* idx4 = m->idx4;
-      if (pipeline == UW_PIPE_TRANSCODE) {
-        if ((st = launch_decode(m, 2, scratch, status, s)) != UW_OK) return st;
-        idx4 = static_cast<const uint8_t*>(scratch);
-      }
-      if (!idx4) return UW_ERR_INVALID_ARG;
+    case UW_PIPE_DIRECT:
+      if (!m->pack || !m->pack_off) return UW_ERR_INVALID_ARG;
+      a.loader = kLoaderPACK;
+      a.pack = m->pack;
+      a.pack_off = m->pack_off;
+      a.vflags = m->vflags;
+      a.vprefix = m->vprefix;
+      a.verbatim = m->verbatim;
+      a.palette = m->cb.palette;
+      a.code_len = m->cb.code_len;
+      break;
+    case UW_PIPE_TRANSCODE: {
+      if ((st = launch_decode(m, 2, scratch, status, s)) != UW_OK) return st;
+      const uint8_t* idx4 = static_cast<const uint8_t*>(scratch);
       a.loader = kLoaderIDX4;
       a.sm = m->sm;
       a.aux = idx4;
@@ -780,13 +994,13 @@ extern "C" uw_status uw_gemm(const uw_matrix* m, int32_t pipeline, const uint16_
 
 extern "C" uw_status uw_gemm_direct_palette(const uw_matrix* m, const uint16_t* x, int32_t batch, uint16_t* y,
                                             void* ws, size_t ws_bytes, void* stream) {
-  if (!m || !m->idx4) return UW_ERR_INVALID_ARG;
+  if (!m || !m->pack || !m->pack_off) return UW_ERR_INVALID_ARG;
   return uw_gemm(m, UW_PIPE_DIRECT, x, batch, y, ws, ws_bytes, stream);
 }
 
 extern "C" uw_status uw_gemm_direct_palette_general_lookup(const uw_matrix* m, const uint16_t* x, int32_t batch,
                                                            uint16_t* y, void* ws, size_t ws_bytes, void* stream) {
-  if (!m || !m->idx4 || !ws) return UW_ERR_INVALID_ARG;
+  if (!m || !m->pack || !m->pack_off || !ws) return UW_ERR_INVALID_ARG;
   return run_pipeline(m, UW_PIPE_DIRECT, x, batch, y, nullptr, ws, ws_bytes, nullptr, 0,
                       static_cast<cudaStream_t>(stream), 1);
 }

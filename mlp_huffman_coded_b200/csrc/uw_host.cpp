@@ -327,3 +327,28 @@ extern "C" const char* uw_status_string(uw_status s) {
 }
 
 extern "C" int32_t uw_version(void) { return 100; }
+
+extern "C" uw_status uw_direct_pack_offsets(const uw_layout* L, const uint32_t* vflags, uint32_t* off,
+                                            uint64_t* pack_bytes) {
+  if (!L || !vflags || !off) return UW_ERR_INVALID_ARG;
+  if (!shape_ok(L->rows, L->cols)) return UW_ERR_UNSUPPORTED_SHAPE;
+  const int64_t kb_n = L->cols / kGroup;
+  const int64_t wpr = (kb_n + 31) / 32;
+  if (L->words_per_row != wpr) return UW_ERR_CORRUPT;
+  const int64_t mt_n = (L->rows + 127) / 128;
+  uint64_t pos = 0;  // 16-byte units
+  int64_t t = 0;
+  for (int64_t mt = 0; mt < mt_n; ++mt) {
+    const int64_t r_end = std::min<int64_t>(L->rows, (mt + 1) * 128);
+    for (int64_t kb = 0; kb < kb_n; ++kb, ++t) {
+      int nv = 0;
+      for (int64_t n = mt * 128; n < r_end; ++n) nv += (vflags[n * wpr + kb / 32] >> (kb % 32)) & 1;
+      off[t] = static_cast<uint32_t>(pos);
+      pos += (12416 + 128 * std::min(nv, 32)) / 16;
+      if (pos >= (uint64_t(1) << 32)) return UW_ERR_UNSUPPORTED_SHAPE;
+    }
+  }
+  off[t] = static_cast<uint32_t>(pos);
+  if (pack_bytes) *pack_bytes = pos * 16;
+  return UW_OK;
+}

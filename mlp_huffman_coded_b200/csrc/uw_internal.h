@@ -61,7 +61,7 @@ uw_status check_matrix(const uw_matrix* m);
 
 // Kernel launchers (asynchronous).
 uw_status launch_decode(const uw_matrix* m, int mode, void* out, uint32_t* status, cudaStream_t s);
-enum Loader { kLoaderBF16 = 0, kLoaderEXP8 = 1, kLoaderIDX4 = 2 };
+enum Loader { kLoaderBF16 = 0, kLoaderEXP8 = 1, kLoaderIDX4 = 2, kLoaderPACK = 3 };
 struct GemmArgs {
   int loader = kLoaderIDX4;
   int64_t N = 0, K = 0;
@@ -73,7 +73,9 @@ struct GemmArgs {
   const uint32_t* vprefix = nullptr;
   const uint16_t* verbatim = nullptr;
   int wpr = 0;
-  const uint8_t* palette = nullptr;   // 16 entries (IDX4 loader)
+  const uint8_t* pack = nullptr;      // direct-palette records (PACK loader)
+  const uint32_t* pack_off = nullptr;
+  const uint8_t* palette = nullptr;   // 16 entries (IDX4 / PACK loaders)
   const uint8_t* code_len = nullptr;  // which palette entries are in use
   const uint16_t* x = nullptr;
   uint16_t* y = nullptr;

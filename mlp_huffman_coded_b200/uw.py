@@ -17,7 +17,8 @@ from dataclasses import dataclass
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libuw.so")
+# UW_LIB_PATH selects another build of the same library (e.g. a tuning build)
+LIB_PATH = os.environ.get("UW_LIB_PATH") or os.path.join(_HERE, "libuw.so")
 
 PIPE_FULL, PIPE_EXPONENT, PIPE_TRANSCODE, PIPE_DIRECT, PIPE_BF16 = 0, 1, 2, 3, 4
 PIPELINES = {"full": PIPE_FULL, "exponent": PIPE_EXPONENT, "transcode": PIPE_TRANSCODE,
@@ -52,7 +53,8 @@ class Layout(C.Structure):
 class Matrix(C.Structure):
     _fields_ = [("L", Layout), ("cb", Codebook), ("sm", C.c_void_p), ("stream", C.c_void_p),
                 ("chunk_bit_off", C.c_void_p), ("vflags", C.c_void_p), ("vprefix", C.c_void_p),
-                ("verbatim", C.c_void_p), ("idx4", C.c_void_p)]
+                ("verbatim", C.c_void_p), ("idx4", C.c_void_p), ("pack", C.c_void_p),
+                ("pack_off", C.c_void_p)]
 
 
 _P = C.c_void_p
@@ -61,6 +63,8 @@ _SIGS = {
     "uw_encode": (C.c_int, [_P, C.c_int64, C.c_int64, C.POINTER(Codebook), C.c_int32, C.POINTER(Layout),
                             _P, _P, _P, _P, _P, _P]),
     "uw_validate": (C.c_int, [C.POINTER(Matrix)]),
+    "uw_direct_pack_offsets": (C.c_int, [C.POINTER(Layout), _P, _P, C.POINTER(C.c_uint64)]),
+    "uw_pack_direct_palette": (C.c_int, [C.POINTER(Matrix), _P, _P, _P]),
     "uw_workspace_bytes": (C.c_size_t, [C.POINTER(Layout), C.c_int32, C.c_int32]),
     "uw_workspace_init": (C.c_int, [_P, C.c_size_t, _P]),
     "uw_workspace_status": (C.c_int, [_P, _P]),
@@ -157,7 +161,18 @@ class HostEncoded:
         m.vflags, m.vprefix = _ptr(self.vflags), _ptr(self.vprefix)
         m.verbatim = _ptr(self.verbatim) if self.verbatim.size else None
         m.idx4 = None
+        m.pack = None
+        m.pack_off = None
         return m
+
+    def pack_offsets(self):
+        """Direct-palette record offsets (16-byte units) and total bytes."""
+        n_tiles = -(-self.rows // 128) * (self.cols // 64)
+        off = np.empty(n_tiles + 1, np.uint32)
+        total = C.c_uint64()
+        _check(lib().uw_direct_pack_offsets(C.byref(self.layout), _ptr(self.vflags), _ptr(off), C.byref(total)),
+               "uw_direct_pack_offsets")
+        return off, int(total.value)
 
     def compressed_bytes(self, form: str = "huffman") -> int:
         meta = self.vflags.nbytes + self.vprefix.nbytes + self.verbatim.nbytes
@@ -251,6 +266,10 @@ class DeviceMatrix:
         self.mat.vflags, self.mat.vprefix = self.vflags.data_ptr(), self.vprefix.data_ptr()
         self.mat.verbatim = self.verbatim.data_ptr() if self.verbatim is not None else None
         self.mat.idx4 = None
+        self.mat.pack = None
+        self.mat.pack_off = None
+        self.pack = None
+        self.pack_off = None
 
     @property
     def rows(self):
@@ -260,18 +279,30 @@ class DeviceMatrix:
     def cols(self):
         return self.enc.cols
 
-    def prepare_direct_palette(self, ws: Workspace, stream=None):
-        """Load-time transcode to 4-bit palette indices (direct palette)."""
+    def prepare_direct_palette(self, ws: Workspace, stream=None, keep_idx4: bool = True):
+        """Load-time preparation of the direct-palette form: transcode to 4-bit
+        palette indices, then gather sm + indices + verbatim rows into one
+        record per 128x64 tile (uw_pack_direct_palette)."""
         import torch
         self.idx4 = torch.empty(self.rows * self.cols // 2, dtype=torch.uint8, device=self.device)
         transcode_palette(self, self.idx4, ws, stream)
         self.mat.idx4 = self.idx4.data_ptr()
+        off, nbytes = self.enc.pack_offsets()
+        self.pack_off = torch.from_numpy(off.view(np.int32)).to(self.device)
+        self.pack = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        _check(lib().uw_pack_direct_palette(C.byref(self.mat), self.pack_off.data_ptr(), self.pack.data_ptr(),
+                                            _stream(stream)), "uw_pack_direct_palette")
+        self.mat.pack = self.pack.data_ptr()
+        self.mat.pack_off = self.pack_off.data_ptr()
+        if not keep_idx4:
+            self.mat.idx4 = None
+            self.idx4 = None
         return self
 
     def direct_palette_bytes(self) -> int:
-        """Bytes the direct-palette GEMM reads from HBM for W."""
-        e = self.enc
-        return (e.sm.nbytes + e.rows * e.cols // 2 + e.vflags.nbytes + e.vprefix.nbytes + e.verbatim.nbytes)
+        """Bytes the direct-palette GEMM reads from HBM for W: the pack
+        records (sm + 4-bit indices + masks + inline verbatim rows)."""
+        return int(self.pack.numel()) if self.pack is not None else 0
 
 
 def workspace_bytes(dm_or_layout, pipeline: int, batch: int) -> int:

@@ -44,7 +44,7 @@ def test_every_declared_symbol_is_exported():
 def test_struct_sizes_match_the_header():
     assert C.sizeof(uw.Codebook) == 200
     assert C.sizeof(uw.Layout) == 64
-    assert C.sizeof(uw.Matrix) == 64 + 200 + 7 * 8
+    assert C.sizeof(uw.Matrix) == 64 + 200 + 9 * 8
 
 
 def test_status_strings_and_version():
@@ -188,3 +188,14 @@ def test_oracle_decodes_the_library_stream():
     ref.stream = enc.stream.copy()
     ref.chunk_bit_off = enc.chunk_bit_off.copy()
     assert np.array_equal(O.decode_full(ref, lockstep=False), w)
+
+
+@pytest.mark.parametrize("rows,cols,rate", [(256, 512, 5e-4), (200, 640, 2e-2), (128, 64, 0.3)])
+def test_direct_pack_offsets_match_oracle(rows, cols, rate):
+    w = synth.weight_matrix(rows, cols, 0.02, rate, 300.0, rows)
+    enc = uw.encode(w)
+    off, total = enc.pack_offsets()
+    ref = O.encode(w)
+    pack, ref_off = O.direct_pack(ref, O.transcode_palette(ref, lockstep=False))
+    assert np.array_equal(off, ref_off)
+    assert total == pack.size == 16 * int(ref_off[-1])

@@ -127,3 +127,13 @@ def test_garbage_stream_stays_in_bounds():
     out = torch.empty(64 * 512, dtype=torch.uint8, device="cuda")
     uw.decode_exponent_only(dm, out, ws)
     assert ws.status() == uw.UW_ERR_CORRUPT
+
+
+@pytest.mark.parametrize("rows,cols,rate", [(256, 512, 5e-4), (200, 640, 2e-2), (384, 4096, 1e-4)])
+def test_direct_pack_bit_exact(rows, cols, rate):
+    w = synth.weight_matrix(rows, cols, 0.02, rate, 300.0, rows + 1)
+    dm = device_matrix(w)
+    ref = O.encode(w)
+    pack, off = O.direct_pack(ref, O.transcode_palette(ref, lockstep=False))
+    assert np.array_equal(dm.pack_off.cpu().numpy().view(np.uint32), off)
+    assert np.array_equal(dm.pack.cpu().numpy(), pack)

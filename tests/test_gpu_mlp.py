@@ -6,7 +6,7 @@ from mlp_huffman_coded_b200 import synth
 from mlp_huffman_coded_b200 import uw
 from oracle import uw_oracle as O
 
-from gpu_util import device_matrix, empty_bf16, to_dev, to_host_u16, within_tol
+from gpu_util import device_matrix, empty_bf16, mlp_check, to_dev, to_host_u16
 
 pytestmark = pytest.mark.gpu
 
@@ -35,14 +35,13 @@ def test_mlp_block_small(B):
     gate, up, down = _block(512, 1536, 61)
     dms = [device_matrix(m) for m in (gate, up, down)]
     x = synth.activations(B, 512, 62)
-    ref = O.mlp_block(gate, up, down, x)
     outs = []
     for pipes in ([3, 3, 3], [0, 1, 2], [2, 3, 0], [1, 1, 1]):
         ws = uw.Workspace(uw.mlp_workspace_bytes(*dms, pipes, B))
         y = empty_bf16(B, 512)
         uw.mlp_block(*dms, pipes, to_dev(x), y, ws)
         ws.check("mlp")
-        ok, err, rms = within_tol(to_host_u16(y), ref)
+        ok, err, rms = mlp_check(to_host_u16(y), gate, up, down, x)
         assert ok, (pipes, err, rms)
         outs.append(to_host_u16(y))
     for o in outs[1:]:
@@ -74,7 +73,7 @@ def test_full_size_mlp_block_batch8():
     y = empty_bf16(8, 4096)
     uw.mlp_block(*dms, [3, 3, 3], to_dev(x), y, ws)
     ws.check()
-    ok, err, rms = within_tol(to_host_u16(y), O.mlp_block(gate, up, down, x))
+    ok, err, rms = mlp_check(to_host_u16(y), gate, up, down, x)
     assert ok, (err, rms)
 
 
@@ -91,7 +90,7 @@ def test_autotune_picks_the_fastest_it_measured():
     assert us.shape == (3, 4) and np.isfinite(us).all() and (us > 0).all()
     for i in range(3):
         assert choice[i] == int(np.argmin(us[i]))
-    # without the load-time transcode, DIRECT is unavailable
-    dm.mat.idx4 = None
+    # without the load-time pack, DIRECT is unavailable
+    dm.mat.pack = None
     choice, us = uw.autotune(dm, [4], 3, x, y, ws)
     assert np.isinf(us[0, 3]) and choice[0] != 3
