@@ -299,6 +299,31 @@ UW_API uw_status uw_gemm_direct_palette_general_lookup(const uw_matrix* m, const
                                                        int32_t batch, uint16_t* y, void* workspace,
                                                        size_t workspace_bytes, void* stream);
 
+/* Direct-palette GEMM for callers that cannot allocate device memory (the
+ * Unweight page has no counterpart; this is a deployment convenience).
+ * Some callers cannot hand the library a workspace -- e.g. an inference
+ * engine that gives a kernel plugin only its input and output buffers
+ * because it plans all device memory ahead of time.  This call computes the
+ * same y as uw_gemm_direct_palette (same kernel, same K split) but keeps the
+ * scratch in a 16 MiB array built into the library, so it allocates nothing
+ * (no cudaMalloc/cudaFree, no allocating library call).
+ *   - Every GPU that loads the library holds that 16 MiB until exit.
+ *   - Limit: header + tile counters + split-K partials must fit in it, i.e.
+ *     (ceil(rows/128)*ceil(batch/256) + SMs) * batch_tile * 512 bytes plus a
+ *     few KB; a 14336 x 4096 matrix fits up to batch 64.  Larger sizes return
+ *     UW_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *   - The first call on a device looks the array's device address up
+ *     (cudaGetSymbolAddress); make that first call before any stream
+ *     capture.
+ *   - Each call zeroes the array's status word and counters on `stream`
+ *     before the kernel; all calls share the one array, so calls that may
+ *     overlap on the GPU (different streams without ordering) race.
+ *   - Device-side problems (a timed-out wait, inconsistent pack offsets) are
+ *     recorded in the array's status word, which this call does not report;
+ *     use uw_gemm_direct_palette with a workspace to diagnose them. */
+UW_API uw_status uw_gemm_direct_palette_noalloc(const uw_matrix* m, const uint16_t* x, int32_t batch,
+                                                uint16_t* y, void* stream);
+
 /* Uncompressed comparator: y = x W^T with W given as device BF16
  * [rows, cols]; the same GEMM kernel, loader reading BF16 tiles.  Workspace:
  * uw_workspace_bytes with UW_PIPE_BF16. */

@@ -74,6 +74,7 @@ _SIGS = {
     "uw_gemm_direct_palette": (C.c_int, [C.POINTER(Matrix), _P, C.c_int32, _P, _P, C.c_size_t, _P]),
     "uw_gemm_direct_palette_general_lookup": (C.c_int, [C.POINTER(Matrix), _P, C.c_int32, _P, _P,
                                                         C.c_size_t, _P]),
+    "uw_gemm_direct_palette_noalloc": (C.c_int, [C.POINTER(Matrix), _P, C.c_int32, _P, _P]),
     "uw_gemm": (C.c_int, [C.POINTER(Matrix), C.c_int32, _P, C.c_int32, _P, _P, C.c_size_t, _P]),
     "uw_gemm_bf16": (C.c_int, [_P, C.c_int64, C.c_int64, _P, C.c_int32, _P, _P, C.c_size_t, _P]),
     "uw_swiglu": (C.c_int, [_P, _P, _P, C.c_int64, _P]),
@@ -333,6 +334,13 @@ def gemm_direct_palette(dm: DeviceMatrix, x, y, ws: Workspace, stream=None, gene
     f = lib().uw_gemm_direct_palette_general_lookup if general_lookup else lib().uw_gemm_direct_palette
     _check(f(C.byref(dm.mat), _ptr(x), x.shape[0], _ptr(y), ws.ptr, ws.nbytes, _stream(stream)),
            "uw_gemm_direct_palette")
+
+
+def gemm_direct_palette_noalloc(dm: DeviceMatrix, x, y, stream=None):
+    """Direct-palette GEMM for callers that cannot allocate: the scratch is
+    the library's own fixed device array (see uw.h)."""
+    _check(lib().uw_gemm_direct_palette_noalloc(C.byref(dm.mat), _ptr(x), x.shape[0], _ptr(y), _stream(stream)),
+           "uw_gemm_direct_palette_noalloc")
 
 
 def gemm_bf16(w, x, y, ws: Workspace, stream=None):
