@@ -51,10 +51,9 @@ constexpr int kWarpProducer = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWarpRebuild0 = 2;
 constexpr int kVCap = 16;         // verbatim rows staged on chip per tile
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 16;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kAccCol = 0;
-constexpr uint32_t kAStageCol0 = 256;
+constexpr uint32_t kAccCol = 0;  // accumulators first; rebuilt A tiles after them
 constexpr size_t kSmemLimit = 227 * 1024;
 constexpr size_t kSmemFloor = 120 * 1024;  // keeps one CTA (and one TMEM owner) per SM
 
@@ -68,6 +67,7 @@ __host__ __device__ constexpr bool loader_pack(int L) { return L == kPACKU || L 
 __host__ __device__ constexpr bool loader_uniform(int L) { return L == kIDX4U || L == kPACKU; }
 constexpr uint32_t kRecIdx = 8192, kRecMask = 12288, kRecVerb = 12416, kRecVCap = 32;
 constexpr uint32_t kRecMax = kRecVerb + kRecVCap * 128;
+constexpr uint32_t kPackMinVCap = 4;  // verbatim rows staged on chip per tile, at least
 
 struct KParams {
   int N, K, B, KB, n_ntiles, ntile;
@@ -97,6 +97,9 @@ struct KParams {
   uint32_t off_rec;   // pack record inside a stage
   uint32_t soff_off;  // shared-memory copy of this CTA's record offsets
   int n_soff;         // its capacity in words
+  uint32_t a_col0;    // first TMEM column of the rebuilt A tiles (32 per stage)
+  uint32_t epi_off;   // epilogue staging: 2 output chunks (+ 2 gate chunks)
+  int tma_out;        // outputs leave through TMA tensor stores (else per element)
 };
 
 struct Bars {
@@ -105,9 +108,11 @@ struct Bars {
   uint64_t empty[kMaxStages];
   uint64_t acc_full[2], acc_empty[2], drain;
   uint64_t meta_full[2];
+  uint64_t gate_full[2];  // fused SwiGLU: gate chunk landed
   uint32_t tmem_base;
   uint32_t abort;
   uint32_t is_last;
+  uint32_t dep_ready;  // the previous kernel on the stream has completed
 };
 
 __device__ __forceinline__ int64_t unit_begin(int64_t c, const KParams& p) {
@@ -217,7 +222,8 @@ __device__ __forceinline__ void rebuild_row(const uint8_t* stage, const KParams&
 template <int L>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wa,
-                const __grid_constant__ CUtensorMap tm_wb, const KParams p) {
+                const __grid_constant__ CUtensorMap tm_wb, const __grid_constant__ CUtensorMap tm_y,
+                const __grid_constant__ CUtensorMap tm_g, const KParams p) {
   constexpr bool kIdx4 = (L == kIDX4U || L == kIDX4M);  // row-major indices + verbatim store
   constexpr bool kPack = loader_pack(L);
   extern __shared__ uint8_t smem_raw[];
@@ -231,6 +237,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   const int G = p.groups;
   const int warp_epi0 = kWarpRebuild0 + 4 * G;
 
+  if (kPack && warp == kWarpProducer) {
+    // this CTA's record offsets: start pulling them into L2 while the CTA
+    // sets up (one 128-byte line per lane and step)
+    const int64_t pt0 = ((u0 / p.KB) / p.n_ntiles) * static_cast<int64_t>(p.KB);
+    const int64_t n_tiles_total = static_cast<int64_t>((p.N + 127) / 128) * p.KB;
+    const int64_t cnt = p.n_soff < n_tiles_total + 1 - pt0 ? p.n_soff : n_tiles_total + 1 - pt0;
+    for (int64_t w = static_cast<int64_t>(lane) * 32; w < cnt; w += 32 * 32) prefetch_l2(p.pack_off + pt0 + w);
+  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&bars->full[s], 1);
@@ -244,8 +258,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     mbar_init(&bars->drain, 1);
     mbar_init(&bars->meta_full[0], 1);
     mbar_init(&bars->meta_full[1], 1);
+    mbar_init(&bars->gate_full[0], 1);
+    mbar_init(&bars->gate_full[1], 1);
     bars->abort = 0;
     bars->is_last = 0;
+    bars->dep_ready = 0;
     mbar_fence_init();
   }
   if (warp == kWarpMma) {
@@ -254,6 +271,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   }
   if (warp == kWarpProducer && lane == 0) {
     prefetch_tensormap(&tm_x);
+    if (p.tma_out) prefetch_tensormap(&tm_y);
+    if (p.tma_out && p.gate) prefetch_tensormap(&tm_g);
     if (!kPack) prefetch_tensormap(&tm_wa);
     if (L != kBF16 && !kPack) prefetch_tensormap(&tm_wb);
   }
@@ -302,12 +321,50 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       const int64_t n_tiles_total = static_cast<int64_t>((p.N + 127) / 128) * p.KB;
       const int64_t want = static_cast<int64_t>(mt_last - mt_first + 1) * p.KB + 1;
       const int64_t cnt = want < p.n_soff ? want : p.n_soff;
-      for (int64_t w = lane; w < cnt; w += 32)
-        soff[w] = (pt_min + w <= n_tiles_total) ? __ldg(p.pack_off + pt_min + w) : 0u;
+      // all loads of a 256-word chunk are in flight before the first store:
+      // one memory round trip per chunk instead of one per word and lane
+      for (int64_t w0 = 0; w0 < cnt; w0 += 256) {
+        uint32_t v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int64_t w = w0 + j * 32 + lane;
+          v[j] = (w < cnt && pt_min + w <= n_tiles_total) ? __ldg(p.pack_off + pt_min + w) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int64_t w = w0 + j * 32 + lane;
+          if (w < cnt) soff[w] = v[j];
+        }
+      }
       __syncwarp();
     }
     int cur_mt = -1;
     int64_t i = 0;
+    const uint64_t stream_policy = l2_evict_first();
+    // Activations may be the output of the previous kernel on the stream
+    // (programmatic dependent launch lets this kernel start while that one
+    // finishes).  Weight copies of the first S stages go out at once; their
+    // activation tiles, which complete the same barriers, follow as soon as
+    // an epilogue thread has seen that kernel complete (dep_ready), at the
+    // latest after the S-th weight copy.
+    bool dep_done = false;
+    int64_t x_next = 0;  // first-use stages whose activation tile is issued
+    int kbx = static_cast<int>(u0 % p.KB);
+    int ntx = static_cast<int>((u0 / p.KB) % p.n_ntiles);
+    auto finish_dependency = [&](int64_t n_issued) {
+      griddep_wait();  // immediate once dep_ready is set; formal ordering
+      dep_done = true;
+      for (; x_next < n_issued; ++x_next) {  // stage x_next, first use
+        if (lane == 0)
+          tma_load_2d(smem + static_cast<size_t>(x_next) * p.stage_bytes + p.off_x, &tm_x, kbx * 64,
+                      ntx * p.ntile, &bars->full[x_next]);
+        if (++kbx == p.KB) {
+          kbx = 0;
+          if (++ntx == p.n_ntiles) ntx = 0;
+        }
+      }
+      __syncwarp();
+    };
     // the loop advances (stage, use) and (row block, batch tile, k-block)
     // incrementally: no division per unit
     int s = 0;
@@ -348,6 +405,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           if (lane == 0) record_status(p.status, UW_ERR_CORRUPT);
           rec_bytes = 0;
         }
+        // verbatim rows past the staged ones are read from HBM by the rebuild
+        if (rec_bytes > kRecVerb + p.vcap * 128u) rec_bytes = kRecVerb + p.vcap * 128u;
         tx = p.x_bytes + rec_bytes;
       }
       int vq_dst[4];
@@ -382,10 +441,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(&bars->full[s], tx);
-        tma_load_2d(stage + p.off_x, &tm_x, kb * 64, nt * p.ntile, &bars->full[s]);
+        if (dep_done) tma_load_2d(stage + p.off_x, &tm_x, kb * 64, nt * p.ntile, &bars->full[s]);
         if (kPack) {
           if (rec_bytes)
-            bulk_load(stage + p.off_rec, p.pack + static_cast<uint64_t>(rec_o0) * 16, rec_bytes, &bars->full[s]);
+            bulk_load_hint(stage + p.off_rec, p.pack + static_cast<uint64_t>(rec_o0) * 16, rec_bytes, &bars->full[s],
+                           stream_policy);
         } else if (L == kIDX4U || L == kIDX4M) {
           tma_load_2d(stage + p.off_wa, &tm_wa, kb * 64, mt * 128, &bars->full[s]);
           tma_load_2d(stage + p.off_wb, &tm_wb, kb * 32, mt * 128, &bars->full[s]);
@@ -403,7 +463,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           if (vq_dst[q] >= 0)
             bulk_load(stage + p.off_verb + vq_dst[q] * 128, p.verbatim + vq_src[q] * 64, 128, &bars->full[s]);
       }
+      if (!dep_done) {
+        const uint32_t ready = __shfl_sync(0xFFFFFFFFu, lane == 0 ? ld_acquire_cta(&bars->dep_ready) : 0u, 0);
+        if (ready || i == S - 1 || u == u1 - 1) finish_dependency(i + 1);
+      }
     }
+    // stopped before the first S stages were issued (an abort): still wait
+    // for the previous kernel, and complete the issued stages' barriers
+    if (!dep_done) finish_dependency(i);
     // drain: the last use of every stage and every issued flag load must land
     // before the CTA can exit (normally already complete)
     if (lane == 0) {
@@ -441,7 +508,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         if (!mbar_wait(&bars->full[s], k & 1, &bars->abort, p.status)) break;
         if (!mbar_wait(&bars->rebuilt[s], k & 1, &bars->abort, p.status)) break;
         tc_fence_after();
-        const uint32_t a_tmem = tmem + kAStageCol0 + static_cast<uint32_t>(s) * 32;
+        const uint32_t a_tmem = tmem + p.a_col0 + static_cast<uint32_t>(s) * 32;
         const uint64_t b_desc = b_desc0 + static_cast<uint64_t>(s) * b_step;
         mma_ts(d_tmem, a_tmem + 0, b_desc + 0, p.idesc, first ? 0u : 1u);
         mma_ts(d_tmem, a_tmem + 8, b_desc + 2, p.idesc, 1u);
@@ -519,7 +586,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           }
         }
       }
-      tmem_st32(tmem + (static_cast<uint32_t>(q * 32) << 16) + kAStageCol0 + static_cast<uint32_t>(s) * 32, o);
+      tmem_st32(tmem + (static_cast<uint32_t>(q * 32) << 16) + p.a_col0 + static_cast<uint32_t>(s) * 32, o);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -527,8 +594,63 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     }
   } else {
     // ------------------------------- epilogue -------------------------------
+    // the outputs, the gate operand and the workspace counters may still be
+    // in use by the previous kernel on the stream until it has completed;
+    // tell the producer (activation loads) and let the next kernel launch
+    griddep_wait();
+    if (warp == warp_epi0 && lane == 0) {
+      st_release_cta(&bars->dep_ready, 1u);
+      griddep_launch_dependents();
+    }
     const int q = warp & 3;
     const int r = q * 32 + lane;
+    const bool elected = warp == warp_epi0 && lane == 0;
+    // Output chunks (16 batch rows x 128 weight rows) are staged in shared
+    // memory as [b][n] bf16 and leave through one TMA tensor store each: two
+    // buffers, one group barrier per chunk.  With the fused SwiGLU the gate
+    // chunk arrives by TMA load into the matching gate buffer, one chunk ahead.
+    __nv_bfloat16* out_s = reinterpret_cast<__nv_bfloat16*>(smem + p.epi_off);
+    __nv_bfloat16* gate_s = out_s + 2 * 16 * 128;
+    const bool tma_gate = p.tma_out && p.gate != nullptr;
+    uint32_t ch = 0;        // output chunks of this CTA so far (buffer ch & 1)
+    uint32_t gate_next = 0;  // gate chunks issued (elected thread)
+    auto load_gate = [&](uint32_t chunk, int mt_, int b0) {
+      gate_next = chunk + 1;
+      uint64_t* gb = &bars->gate_full[chunk & 1];
+      mbar_arrive_expect_tx(gb, 16u * 128u * 2u);
+      tma_load_2d(gate_s + (chunk & 1) * 16 * 128, &tm_g, mt_ * 128, b0, gb);
+    };
+    // one chunk of final values acc[jj] = y[b0 + jj][n]
+    auto emit = [&](const float (&acc)[16], int mt_, int b0, int64_t n, bool row_ok) -> bool {
+      if (!p.tma_out) {
+        if (row_ok) {
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj)
+            if (b0 + jj < p.B) store_out(p, b0 + jj, n, acc[jj]);
+        }
+        return true;
+      }
+      __nv_bfloat16* os = out_s + (ch & 1) * 16 * 128 + r;
+      if (tma_gate) {
+        const bool got = mbar_wait(&bars->gate_full[ch & 1], (ch >> 1) & 1, &bars->abort, p.status);
+        if (!group_and(got)) return false;
+        const __nv_bfloat16* gs = gate_s + (ch & 1) * 16 * 128 + r;
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) os[jj * 128] = swiglu_bf16(gs[jj * 128], __float2bfloat16_rn(acc[jj]));
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) os[jj * 128] = __float2bfloat16_rn(acc[jj]);
+      }
+      fence_proxy_async_smem();
+      if (elected) bulk_wait_group_read0();  // the other buffer's store has read its data
+      group_sync();
+      if (elected) {
+        tma_store_2d(&tm_y, out_s + (ch & 1) * 16 * 128, mt_ * 128, b0);
+        bulk_commit_group();
+      }
+      ++ch;
+      return true;
+    };
     uint32_t seg = 0;
     int64_t u = u0;
     while (u < u1) {
@@ -539,6 +661,18 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       const int64_t c_first = unit_owner(t * p.KB, p);
       const int64_t c_last = unit_owner(t * p.KB + p.KB - 1, p);
       const int ncontrib = static_cast<int>(c_last - c_first + 1);
+      // A tile split over several CTAs is finished by the first of them
+      // (c_first): its part is the first k-blocks of the tile, the last
+      // segment of its range, so the other contributors (their parts open
+      // their ranges) have normally published long before.  It keeps its own
+      // sums in TMEM, adds the others' partials in CTA order and stores y.
+      // The others write partials and publish them with one release add.
+      const bool reducer = ncontrib > 1 && blockIdx.x == c_first;
+      const bool out_seg = ncontrib == 1 || reducer;
+      const int b_first = nt * p.ntile;
+      // output chunks past the batch are skipped (TMA would clip them anyway)
+      const int n_chunks = out_seg ? min(p.ntile, ((p.B - b_first + 15) / 16) * 16) / 16 : p.ntile / 16;
+      if (out_seg && tma_gate && elected && n_chunks > 0) load_gate(ch, mt, b_first);
       const uint32_t ab = seg % p.n_acc, use = seg / p.n_acc;
       bool ok = mbar_wait(&bars->acc_full[ab], use & 1, &bars->abort, p.status);
       ok = __all_sync(0xFFFFFFFFu, ok);
@@ -549,85 +683,102 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       const bool row_ok = n < p.N;
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + kAccCol + ab * static_cast<uint32_t>(p.ntile);
       const int64_t slot0 = t + c_first;
-      // partial sums: slot-major, then row, then column, so one thread owns a
-      // contiguous run of ntile floats and moves it with 16-byte accesses
+      bool staged = false;
+      if (reducer) {
+        bool got = true;
+        if (elected) {
+          const uint64_t w0 = globaltimer_ns();
+          for (uint32_t it = 0; ld_acquire_gpu(p.counters + t) < static_cast<uint32_t>(ncontrib - 1); ++it) {
+            if ((it & 15) == 15) {
+              if (bars->abort) { got = false; break; }
+              if (globaltimer_ns() - w0 > kWaitLimitNs) {
+                record_status(p.status, UW_ERR_TIMEOUT);
+                bars->abort = 1;
+                got = false;
+                break;
+              }
+            }
+            __nanosleep(100);
+          }
+        }
+        if (!group_and(got)) break;  // also orders the partial loads after the acquire
+        // on the CTA's last segment every stage has been consumed: copy the
+        // other partials of this thread's row into the stage buffers at once
+        // (one round trip), when they fit
+        staged = seg_end == u1 && static_cast<uint64_t>(S) * p.stage_bytes >=
+                                      static_cast<uint64_t>(ncontrib - 1) * 512u * static_cast<uint32_t>(p.ntile);
+        if (staged) {
+          float* stg = reinterpret_cast<float*>(smem);
+          for (int jc = 1; jc < ncontrib; ++jc) {
+            const float* src = p.partials + ((slot0 + jc) * 128 + r) * p.ntile;
+            float* dst = stg + (static_cast<size_t>(jc - 1) * 128 + r) * p.ntile;
+            for (int f = 0; f < n_chunks * 16; f += 4) cp_async_16(dst + f, src + f);
+          }
+          cp_async_wait_all();
+        }
+      }
       float* my_part = p.partials + ((slot0 + (blockIdx.x - c_first)) * 128 + r) * p.ntile;
-      for (int cc = 0; cc < p.ntile / 16; ++cc) {
+      for (int cc = 0; cc < n_chunks && ok; ++cc) {
         uint32_t v[16];
         tmem_ld16(taddr + cc * 16, v);
         tc_wait_ld();
-        if (ncontrib == 1) {
-          if (row_ok) {
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-              const int b = nt * p.ntile + cc * 16 + jj;
-              if (b < p.B) store_out(p, b, n, __uint_as_float(v[jj]));
-            }
-          }
-        } else {
+        if (!out_seg) {
           float4* dst = reinterpret_cast<float4*>(my_part + cc * 16);
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4)
             dst[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
                                   __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
+          continue;
         }
+        float acc[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) acc[jj] = __uint_as_float(v[jj]);
+        if (reducer) {
+          // the other contributors' partials of these 16 columns, CTA order
+          for (int jc = 1; jc < ncontrib; ++jc) {
+            const float4* src =
+                staged ? reinterpret_cast<const float4*>(reinterpret_cast<const float*>(smem) +
+                                                         (static_cast<size_t>(jc - 1) * 128 + r) * p.ntile + cc * 16)
+                       : reinterpret_cast<const float4*>(p.partials + ((slot0 + jc) * 128 + r) * p.ntile + cc * 16);
+            float4 w4[4];
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) w4[q4] = staged ? src[q4] : __ldcg(src + q4);
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              acc[4 * q4] += w4[q4].x;
+              acc[4 * q4 + 1] += w4[q4].y;
+              acc[4 * q4 + 2] += w4[q4].z;
+              acc[4 * q4 + 3] += w4[q4].w;
+            }
+          }
+        }
+        if (!emit(acc, mt, b_first + cc * 16, n, row_ok)) {
+          ok = false;
+          break;
+        }
+        if (tma_gate && elected && cc + 1 < n_chunks) load_gate(ch, mt, b_first + (cc + 1) * 16);
       }
+      if (!ok) break;
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);
       if (ncontrib > 1) {
-        __threadfence();
-        group_sync();
-        if (warp == warp_epi0 && lane == 0) {
-          const uint32_t old = atomicAdd(p.counters + t, 1u);
-          bars->is_last = (old == static_cast<uint32_t>(ncontrib - 1)) ? 1u : 0u;
-        }
-        group_sync();
-        if (bars->is_last) {
-          __threadfence();
-          // fixed order: contributor 0, 1, ... (the CTA order), independent of
-          // which CTA finished last; 16 columns at a time, all loads of a
-          // chunk issued before any is summed
-          for (int cc = 0; cc < p.ntile / 16; ++cc) {
-            float acc[16];
-#pragma unroll
-            for (int jj = 0; jj < 16; ++jj) acc[jj] = 0.0f;
-            for (int jc = 0; jc < ncontrib; jc += 4) {
-              float4 ld[4][4];
-#pragma unroll
-              for (int a = 0; a < 4; ++a)
-                if (jc + a < ncontrib) {
-                  const float4* src = reinterpret_cast<const float4*>(
-                      p.partials + ((slot0 + jc + a) * 128 + r) * p.ntile + cc * 16);
-#pragma unroll
-                  for (int q4 = 0; q4 < 4; ++q4) ld[a][q4] = __ldcg(src + q4);
-                }
-#pragma unroll
-              for (int a = 0; a < 4; ++a)
-                if (jc + a < ncontrib) {
-#pragma unroll
-                  for (int q4 = 0; q4 < 4; ++q4) {
-                    acc[4 * q4] += ld[a][q4].x;
-                    acc[4 * q4 + 1] += ld[a][q4].y;
-                    acc[4 * q4 + 2] += ld[a][q4].z;
-                    acc[4 * q4 + 3] += ld[a][q4].w;
-                  }
-                }
-            }
-            if (row_ok) {
-#pragma unroll
-              for (int jj = 0; jj < 16; ++jj) {
-                const int b = nt * p.ntile + cc * 16 + jj;
-                if (b < p.B) store_out(p, b, n, acc[jj]);
-              }
-            }
-          }
-          if (warp == warp_epi0 && lane == 0) p.counters[t] = 0;
+        group_sync();  // every partial store of the group precedes the publish
+        if (elected) {
+          if (reducer)
+            p.counters[t] = 0;  // ready for the next launch on this workspace
+          else
+            red_release_gpu_add(p.counters + t, 1u);
         }
       }
       ++seg;
       u = seg_end;
     }
+    // the CTA's shared memory must outlive the copies touching it: gate
+    // chunks still in flight after an abort, and the output stores
+    if (elected && tma_gate)
+      for (uint32_t c = ch; c < gate_next; ++c) mbar_wait(&bars->gate_full[c & 1], (c >> 1) & 1, nullptr, p.status);
+    if (elected && p.tma_out) bulk_wait_group0();
   }
 
   tc_fence_before();
@@ -651,7 +802,7 @@ struct Layout {
   int stages = 0;
   uint32_t stage_bytes = 0, off_x = 0, off_wa = 0, off_wb = 0, off_verb = 0, off_hdr = 0, off_rec = 0;
   uint32_t x_bytes = 0, wa_bytes = 0, wb_bytes = 0;
-  uint32_t meta_off = 0, meta_slot_words = 0, bar_off = 0, soff_off = 0;
+  uint32_t meta_off = 0, meta_slot_words = 0, bar_off = 0, soff_off = 0, a_col0 = 0, epi_off = 0;
   int n_soff = 0, vcap = 0;
   size_t smem = 0;
 };
@@ -680,8 +831,13 @@ int rebuild_groups() {
 
 // Shared-memory plan of one launch.  Every tile region starts on a 1024-byte
 // boundary (the 128-byte swizzle of the activation tile repeats every 1024).
-bool make_layout(int loader, const GemmPlan& plan, int wpr, Layout* out) {
+bool make_layout(int loader, const GemmPlan& plan, int wpr, bool tma_out, bool gate, Layout* out) {
   Layout l;
+  // TMEM: accumulators (n_acc x ntile columns), then one 32-column A tile per
+  // stage
+  const int n_acc = 2 * plan.ntile <= 256 ? 2 : 1;
+  l.a_col0 = (static_cast<uint32_t>(n_acc * plan.ntile) + 31u) & ~31u;
+  const int tmem_stages = static_cast<int>((kTmemCols - l.a_col0) / 32u);
   l.x_bytes = static_cast<uint32_t>(plan.ntile) * 128;
   const bool idx4 = loader == kIDX4U || loader == kIDX4M;
   const bool pack = loader_pack(loader);
@@ -692,8 +848,8 @@ bool make_layout(int loader, const GemmPlan& plan, int wpr, Layout* out) {
     l.off_wb = l.off_rec + kRecIdx;
     l.off_hdr = l.off_rec + kRecMask;
     l.off_verb = l.off_rec + kRecVerb;
-    l.vcap = kRecVCap;
-    l.stage_bytes = a1024(l.off_rec + kRecMax);
+    l.vcap = kRecVCap;  // final value below, from the stage count
+    l.stage_bytes = a1024(l.off_rec + kRecVerb + kPackMinVCap * 128u);
   } else {
     l.wa_bytes = loader == kBF16 ? 16384u : 8192u;
     l.wb_bytes = loader == kBF16 ? 0u : (loader == kEXP8 ? 8192u : 4096u);
@@ -715,23 +871,34 @@ bool make_layout(int loader, const GemmPlan& plan, int wpr, Layout* out) {
     l.n_soff = static_cast<int>(span * plan.KB + 1);
   }
   const uint32_t soff_bytes = a1024(static_cast<uint32_t>(l.n_soff) * 4u);
-  const uint32_t fixed = meta_bytes + soff_bytes + a1024(sizeof(Bars)) + 1024u;  // + alignment slack
+  // epilogue staging: two 16x128 bf16 output chunks, two gate chunks
+  const uint32_t epi_bytes = tma_out ? (gate ? 16384u : 8192u) : 0u;
+  const uint32_t fixed = meta_bytes + soff_bytes + epi_bytes + a1024(sizeof(Bars)) + 1024u;  // + alignment slack
   if (fixed >= kSmemLimit) return false;
   int stages = static_cast<int>((kSmemLimit - fixed) / l.stage_bytes);
-  stages = std::min(stages, max_stages());
+  stages = std::min({stages, max_stages(), tmem_stages});
   if (stages < 2) return false;
   l.stages = stages;
+  if (pack) {
+    // pack records: spread the remaining shared memory over the stages as
+    // on-chip verbatim rows (most tiles have a few; the rest come from HBM)
+    const uint32_t per_stage = ((kSmemLimit - fixed) / static_cast<uint32_t>(stages)) & ~1023u;
+    const uint32_t room = (per_stage - l.off_rec - kRecVerb) / 128u;
+    l.vcap = static_cast<int>(std::min<uint32_t>(room, kRecVCap));
+    l.stage_bytes = a1024(l.off_rec + kRecVerb + static_cast<uint32_t>(l.vcap) * 128u);
+  }
   l.meta_off = static_cast<uint32_t>(stages) * l.stage_bytes;
   l.soff_off = l.meta_off + meta_bytes;
-  l.bar_off = l.soff_off + soff_bytes;
+  l.epi_off = l.soff_off + soff_bytes;
+  l.bar_off = l.epi_off + epi_bytes;
   l.smem = std::max<size_t>(static_cast<size_t>(l.bar_off) + a1024(sizeof(Bars)) + 1024u, kSmemFloor);
   *out = l;
   return true;
 }
 
 template <int L>
-uw_status launch_kernel(const CUtensorMap& x, const CUtensorMap& wa, const CUtensorMap& wb, const KParams& kp,
-                        size_t smem, cudaStream_t s) {
+uw_status launch_kernel(const CUtensorMap& x, const CUtensorMap& wa, const CUtensorMap& wb, const CUtensorMap& y,
+                        const CUtensorMap& g, const KParams& kp, size_t smem, cudaStream_t s) {
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   int dev = 0;
@@ -741,8 +908,23 @@ uw_status launch_kernel(const CUtensorMap& x, const CUtensorMap& wa, const CUten
                                               static_cast<int>(kSmemLimit));
   });
   if (attr_err[dev & 63] != cudaSuccess) return UW_ERR_CUDA;
-  gemm_kernel<L><<<kp.grid, 32 * (6 + 4 * kp.groups), smem, s>>>(x, wa, wb, kp);
+  // programmatic dependent launch: the kernel may start while the previous
+  // kernel on the stream finishes; it streams weights first and waits for
+  // that kernel (griddepcontrol.wait) before reading activations or writing
+  // outputs
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(kp.grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(32 * (6 + 4 * kp.groups)));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t launch_err = cudaLaunchKernelEx(&cfg, gemm_kernel<L>, x, wa, wb, y, g, kp);
   note_launch();
+  if (launch_err != cudaSuccess) return cuda_status(launch_err);
   return cuda_status(cudaGetLastError());
 }
 
@@ -805,11 +987,24 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
     pal = palette_tables(a.palette, a.code_len, &mixed);
     kl = (mixed || a.force_mixed_palette) ? kIDX4M : kIDX4U;
   }
+  // outputs (and the SwiGLU gate) as [B][N] bf16 tensors for TMA: rows must
+  // be 16-byte multiples and the bases 16-byte aligned, else per-element stores
+  const bool tma_out = (a.N % 8) == 0 && aligned16(a.y) && (!a.gate || aligned16(a.gate));
   Layout lay;
-  if (!make_layout(kl, plan, a.wpr, &lay)) return UW_ERR_UNSUPPORTED_SHAPE;
+  if (!make_layout(kl, plan, a.wpr, tma_out, a.gate != nullptr, &lay)) return UW_ERR_UNSUPPORTED_SHAPE;
 
-  CUtensorMap tx, twa, twb;
+  CUtensorMap tx, twa, twb, ty, tg;
   std::memset(&twb, 0, sizeof(twb));
+  std::memset(&ty, 0, sizeof(ty));
+  std::memset(&tg, 0, sizeof(tg));
+  if (tma_out) {
+    if ((st = make_tensor_map_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.y, a.N, a.B, a.N * 2, 128, 16,
+                                 CU_TENSOR_MAP_SWIZZLE_NONE)) != UW_OK)
+      return st;
+    if (a.gate && (st = make_tensor_map_2d(&tg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.gate, a.N, a.B, a.N * 2, 128,
+                                           16, CU_TENSOR_MAP_SWIZZLE_NONE)) != UW_OK)
+      return st;
+  }
   if ((st = make_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, a.K, a.B, a.K * 2, 64, plan.ntile,
                                CU_TENSOR_MAP_SWIZZLE_128B)) != UW_OK)
     return st;
@@ -877,14 +1072,17 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.off_rec = lay.off_rec;
   kp.soff_off = lay.soff_off;
   kp.n_soff = lay.n_soff;
+  kp.a_col0 = lay.a_col0;
+  kp.epi_off = lay.epi_off;
+  kp.tma_out = tma_out ? 1 : 0;
 
   switch (kl) {
-    case kBF16: return launch_kernel<kBF16>(tx, twa, twb, kp, lay.smem, s);
-    case kEXP8: return launch_kernel<kEXP8>(tx, twa, twb, kp, lay.smem, s);
-    case kIDX4U: return launch_kernel<kIDX4U>(tx, twa, twb, kp, lay.smem, s);
-    case kIDX4M: return launch_kernel<kIDX4M>(tx, twa, twb, kp, lay.smem, s);
-    case kPACKU: return launch_kernel<kPACKU>(tx, twa, twb, kp, lay.smem, s);
-    default: return launch_kernel<kPACKM>(tx, twa, twb, kp, lay.smem, s);
+    case kBF16: return launch_kernel<kBF16>(tx, twa, twb, ty, tg, kp, lay.smem, s);
+    case kEXP8: return launch_kernel<kEXP8>(tx, twa, twb, ty, tg, kp, lay.smem, s);
+    case kIDX4U: return launch_kernel<kIDX4U>(tx, twa, twb, ty, tg, kp, lay.smem, s);
+    case kIDX4M: return launch_kernel<kIDX4M>(tx, twa, twb, ty, tg, kp, lay.smem, s);
+    case kPACKU: return launch_kernel<kPACKU>(tx, twa, twb, ty, tg, kp, lay.smem, s);
+    default: return launch_kernel<kPACKM>(tx, twa, twb, ty, tg, kp, lay.smem, s);
   }
 }
 
