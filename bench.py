@@ -35,10 +35,27 @@ D_MODEL, FFN = 4096, 14336
 SIGMA, OUTLIER_RATE, OUTLIER_SCALE, SEED = 0.02, 1e-4, 100.0, 2
 HBM_FALLBACK_GBS = 6650.0
 
-# DRAM traffic (read + write bytes) per launch of the direct-palette GEMM
-# kernel from ncu (see profiles/); None until a capture of the current kernel
-# exists.
-NCU_TRAFFIC_PER_LAUNCH = None
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch
+# of the direct-palette GEMM kernel (the 14336x4096 gate projection at batch 8,
+# ncu --set full; profiles/gemm_direct_palette_14336x4096_b8.md), valid only
+# for the kernel sources it was taken on: reported as null once they change.
+NCU_TRAFFIC = {"bytes_per_launch": 94127104,
+               "launch": "gate projection 14336x4096, batch 8",
+               "sources_sha256": "7457d830303467e8f1c709171d999d83effeb4fc0f190b0ce26a34f781f37ddb"}
+GEMM_SOURCES = ["mlp_huffman_coded_b200/csrc/uw_gemm.cu", "mlp_huffman_coded_b200/csrc/uw_device.cuh",
+                "mlp_huffman_coded_b200/csrc/uw_internal.h"]
+
+
+def ncu_traffic_per_launch():
+    import hashlib
+    h = hashlib.sha256()
+    try:
+        for f in GEMM_SOURCES:
+            with open(os.path.join(ROOT, f), "rb") as fh:
+                h.update(fh.read())
+    except OSError:
+        return None
+    return NCU_TRAFFIC["bytes_per_launch"] if h.hexdigest() == NCU_TRAFFIC["sources_sha256"] else None
 
 
 def measured_peaks():
@@ -349,8 +366,10 @@ def run_gpu(args, world, rank, local):
             "data": "synthetic",
             "config": dict(config_dict(args), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": NCU_TRAFFIC_PER_LAUNCH,
-                         "kernel": "gemm_kernel<IDX4 uniform palette> (3 launches per step)",
+                         "frac": achieved / peak, "traffic": ncu_traffic_per_launch(),
+                         "traffic_launch": NCU_TRAFFIC["launch"],
+                         "kernel": "gemm_kernel<PACK, uniform palette> (direct palette; 3 launches per step, "
+                                   "achieved = algorithmic bytes per step / step time)",
                          "algorithmic_bytes_per_step": per_step_bytes, "peak_source": f"{src} hbm_gbs"},
             "effective_weight_gbs": weight_gbs,
             "bf16_torch_matmul_ms_per_step": bf16_ms,
