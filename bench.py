@@ -68,7 +68,7 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle reasons sampled every 200 ms in the background."""
+    """nvidia-smi clocks/throttle reasons sampled every 50 ms in the background."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -84,7 +84,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except Exception:
             self.proc = None
             return self
@@ -115,7 +115,7 @@ class ClockSampler:
         window = "timed region"
         if not inside:
             inside = rows
-            window = "whole run (timed region shorter than the 200 ms sampling interval)"
+            window = "whole run (timed region shorter than the 50 ms sampling interval)"
         if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "window": "unavailable"}
         sm = [float(p[1]) for _, p in inside if p[1].replace(".", "").isdigit()]
@@ -447,8 +447,9 @@ def run_gemm_case(args, local):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: 3000 GPU steps, ~0.3 s; 20 oracle samples for --impl reference)")
+    ap.add_argument("--warmup", type=int, default=None, help="untimed steps (default 20; 3 for --impl reference)")
     ap.add_argument("--batch", type=int, default=8)
     ap.add_argument("--impl", default="uw", choices=["uw", "reference"])
     ap.add_argument("--ref-fraction", type=float, default=1 / 16)
@@ -458,6 +459,10 @@ def main(argv=None):
     ap.add_argument("--pipeline", default="direct", choices=["full", "exponent", "transcode", "direct", "bf16"])
     ap.add_argument("--no-flush", action="store_true", help="gemm case: leave L2 warm between calls")
     args = ap.parse_args(argv)
+    if args.steps is None:
+        args.steps = 20 if args.impl == "reference" else (100 if args.case == "gemm" else 3000)
+    if args.warmup is None:
+        args.warmup = 3 if args.impl == "reference" else 20
     world, rank, local = dist_init()
     try:
         if args.impl == "reference":
