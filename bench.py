@@ -444,6 +444,104 @@ def run_gemm_case(args, local):
     return 0
 
 
+def _timed(call, flush, steps, warmup, dev):
+    """Median / min µs of `call` over `steps` runs, L2 flushed (clean read of a
+    256 MB buffer) before each, CUDA events on the current stream."""
+    import torch
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize(dev)
+    times = []
+    for _ in range(steps):
+        flush.view(torch.int32).max()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3)
+    return float(np.median(times)), float(np.min(times))
+
+
+def run_decode_case(args, local):
+    """The three preprocessing decoders on the 14336x4096 gate-shaped matrix
+    (sigma 0.02, 1e-4 outliers x100, seed 1): µs, GB/s of compressed input
+    read and of output written, and (read + write) / time against HBM."""
+    import torch
+    from mlp_huffman_coded_b200 import synth, uw
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.weight_matrix(FFN, D_MODEL, SIGMA, OUTLIER_RATE, OUTLIER_SCALE, seed=1)
+    enc = uw.encode(w)
+    dm = uw.DeviceMatrix(enc, device=dev)
+    ws = uw.Workspace(256, device=dev)
+    flush = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+    n = w.size
+    meta = enc.chunk_bit_off.nbytes + enc.vflags.nbytes + enc.vprefix.nbytes
+    stream = enc.stream.nbytes
+    verb = enc.verbatim.nbytes
+    peaks, src = measured_peaks()
+    hbm = peaks.get("hbm_gbs", HBM_FALLBACK_GBS)
+    cases = [
+        ("full", torch.empty(n, dtype=torch.int16, device=dev), uw.decode_full, enc.sm.nbytes + stream + meta + verb, 2 * n),
+        ("exponent", torch.empty(n, dtype=torch.uint8, device=dev), uw.decode_exponent_only, stream + meta + verb, n),
+        ("transcode", torch.empty(n // 2, dtype=torch.uint8, device=dev), uw.transcode_palette, stream + meta, n // 2),
+    ]
+    for name, out, fn, rd, wr in cases:
+        med, mn = _timed(lambda: fn(dm, out, ws), flush, args.steps, args.warmup, dev)
+        ws.check(f"decode {name}")
+        print(json.dumps({"case": "decode", "decoder": name, "matrix": "14336x4096 seed 1", "median_us": med,
+                          "min_us": mn, "read_bytes": rd, "write_bytes": wr, "read_gbs": rd / med / 1e3,
+                          "write_gbs": wr / med / 1e3, "hbm_frac": (rd + wr) / med / 1e3 / hbm,
+                          "hbm_peak_gbs": hbm, "peak_source": src}), flush=True)
+    return 0
+
+
+def run_sweep_case(args, local):
+    """SwiGLU block matrices x batch 1..512: the four pipelines, the library's
+    own BF16 GEMM and torch.matmul BF16 (cuBLAS), L2 flushed before each call;
+    then the autotuner's choice per matrix and batch."""
+    import torch
+    from mlp_huffman_coded_b200 import synth, uw
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    batches = [1, 2, 4, 8, 16, 32, 64, 128, 256, 512]
+    mats = synth.mlp_block(D_MODEL, FFN, SIGMA, OUTLIER_RATE, OUTLIER_SCALE, SEED)
+    names = ["gate", "up", "down"]
+    flush = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+    ws0 = uw.Workspace(256, device=dev)
+    for name, w in zip(names, mats):
+        dm = uw.DeviceMatrix(uw.encode(w), device=dev).prepare_direct_palette(ws0)
+        ws0.check("prepare")
+        N, K = w.shape
+        wd = torch.from_numpy(w.view(np.int16)).to(dev)
+        wt = wd.view(torch.bfloat16)
+        ws = uw.Workspace(max(max(uw.workspace_bytes(dm, p, max(batches)) for p in range(4)),
+                              uw.workspace_bytes(dm, uw.PIPE_BF16, max(batches))), device=dev)
+        xall = torch.from_numpy(synth.activations(max(batches), K, 3).view(np.int16)).to(dev)
+        for B in batches:
+            x = xall[:B].contiguous()
+            y = torch.empty(B, N, dtype=torch.int16, device=dev)
+            row = {"case": "sweep", "matrix": f"{name} {N}x{K}", "batch": B}
+            for pname, pipe in (("full", uw.PIPE_FULL), ("exponent", uw.PIPE_EXPONENT),
+                                ("transcode", uw.PIPE_TRANSCODE), ("direct", uw.PIPE_DIRECT)):
+                row[pname + "_us"] = _timed(lambda: uw.gemm(dm, pipe, x, y, ws), flush, args.steps, args.warmup, dev)[0]
+            row["own_bf16_us"] = _timed(lambda: uw.gemm_bf16(wd, x, y, ws), flush, args.steps, args.warmup, dev)[0]
+            xb = x.view(torch.bfloat16)
+            row["torch_bf16_us"] = _timed(lambda: xb @ wt.T, flush, args.steps, args.warmup, dev)[0]
+            ws.check("sweep")
+            print(json.dumps(row), flush=True)
+        y = torch.empty(max(batches), N, dtype=torch.int16, device=dev)
+        choice, us = uw.autotune(dm, batches, max(3, args.steps // 2), xall, y, ws, flush=flush)
+        ws.check("autotune")
+        print(json.dumps({"case": "autotune", "matrix": f"{name} {N}x{K}", "batches": batches,
+                          "choice": [["full", "exponent", "transcode", "direct"][c] for c in choice],
+                          "us": np.round(us, 2).tolist()}), flush=True)
+        del dm, wd, ws
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -454,21 +552,26 @@ def main(argv=None):
     ap.add_argument("--impl", default="uw", choices=["uw", "reference"])
     ap.add_argument("--ref-fraction", type=float, default=1 / 16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", default="block", choices=["block", "gemm"],
-                    help="gemm: one 14336x4096 matrix through --pipeline (profiling unit)")
+    ap.add_argument("--case", default="block", choices=["block", "gemm", "decode", "sweep"],
+                    help="gemm: one 14336x4096 matrix through --pipeline (profiling unit); decode: the three "
+                         "decoders on it; sweep: pipelines x batch 1..512 x block matrices + autotune")
     ap.add_argument("--pipeline", default="direct", choices=["full", "exponent", "transcode", "direct", "bf16"])
     ap.add_argument("--no-flush", action="store_true", help="gemm case: leave L2 warm between calls")
     args = ap.parse_args(argv)
     if args.steps is None:
-        args.steps = 20 if args.impl == "reference" else (100 if args.case == "gemm" else 3000)
+        args.steps = 20 if args.impl == "reference" else {"gemm": 100, "decode": 20, "sweep": 10}.get(args.case, 3000)
     if args.warmup is None:
-        args.warmup = 3 if args.impl == "reference" else 20
+        args.warmup = 3 if args.impl == "reference" or args.case in ("sweep", "decode") else 20
     world, rank, local = dist_init()
     try:
         if args.impl == "reference":
             return run_reference(args, world, rank)
         if args.case == "gemm":
             return run_gemm_case(args, local)
+        if args.case == "decode":
+            return run_decode_case(args, local)
+        if args.case == "sweep":
+            return run_sweep_case(args, local)
         return run_gpu(args, world, rank, local)
     finally:
         if world > 1:
