@@ -58,6 +58,7 @@ struct DecodeTables {
   uint32_t count[17];      // codes of each length
   uint32_t offset[17];     // index of the first symbol of each length
   uint8_t sorted[16];      // symbols in (length, index) order
+  uint8_t palette[16];
 };
 
 __device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables& t) {
@@ -76,6 +77,7 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables
     for (int l = 1; l <= 15; ++l)
       for (int i = 0; i < 16; ++i)
         if (p.code_len[i] == l) t.sorted[k++] = static_cast<uint8_t>(i);
+    for (int i = 0; i < 16; ++i) t.palette[i] = p.palette[i];
   }
   __syncthreads();
   const int lim = p.max_len < kLutBits ? p.max_len : kLutBits;
@@ -95,33 +97,35 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables
   __syncthreads();
 }
 
-// One canonical symbol from the top of a left-aligned 64-bit window.  Returns
-// the LUT-style entry; on an invalid code records UW_ERR_CORRUPT and returns a
-// length-1 entry so decoding stays bounded.
-__device__ __forceinline__ uint32_t decode_one(const DecodeTables& t, const DecodeParams& p,
-                                               uint64_t win) {
-  uint32_t ent = t.lut[static_cast<uint32_t>(win >> (64 - kLutBits))];
-  if (((ent >> 4) & 15) == 0) {
-    ent = 0;
-    for (int l = kLutBits + 1; l <= p.max_len; ++l) {
-      const uint32_t code = static_cast<uint32_t>(win >> (64 - l));
-      const uint32_t d = code - t.first[l];
-      if (t.count[l] && d < t.count[l]) {
-        const int sym = t.sorted[t.offset[l] + d];
-        ent = static_cast<uint32_t>(sym | (l << 4) | (p.palette[sym] << 8));
-        break;
-      }
-    }
-    if (ent == 0) {
-      record_status(p.status, UW_ERR_CORRUPT);
-      ent = 1u << 4;
+// Codes longer than the table (rare: the tail of the exponent distribution)
+// by canonical first-code comparison.  Out of line: the symbol loop inlines
+// the table path dozens of times and this loop would bloat every copy.
+// On an invalid code records UW_ERR_CORRUPT and returns a length-1 entry so
+// decoding stays bounded.
+__device__ __forceinline__ uint32_t decode_long(const DecodeTables& t, int max_len, uint32_t* status,
+                                             uint64_t win) {
+  for (int l = kLutBits + 1; l <= max_len; ++l) {
+    const uint32_t code = static_cast<uint32_t>(win >> (64 - l));
+    const uint32_t d = code - t.first[l];
+    if (t.count[l] && d < t.count[l]) {
+      const int sym = t.sorted[t.offset[l] + d];
+      return static_cast<uint32_t>(sym | (l << 4) | (t.palette[sym] << 8));
     }
   }
-  return ent;
+  record_status(status, UW_ERR_CORRUPT);
+  return 1u << 4;
+}
+
+// One canonical symbol from the top of a left-aligned 64-bit window, as a
+// table entry (sym | len << 4 | exponent << 8).
+__device__ __forceinline__ uint32_t decode_one(const DecodeTables& t, const DecodeParams& p,
+                                               uint64_t win) {
+  const uint32_t ent = t.lut[static_cast<uint32_t>(win >> (64 - kLutBits))];
+  return ((ent >> 4) & 15) != 0 ? ent : decode_long(t, p.max_len, p.status, win);
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kDecodeThreads, 7) decode_kernel(const DecodeParams p) {
   __shared__ DecodeTables t;
   build_tables(p, t);
   const int64_t last_word = p.stream_words - 1;
@@ -180,14 +184,13 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
         }
         continue;
       }
-      uint4 smv[4];
-      if (MODE == kFull) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.sm + e0);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) smv[k] = __ldg(src + k);
-      }
-#pragma unroll
+      // quarters of 16 symbols, not unrolled (code size: the instruction
+      // cache, not arithmetic, limited the fully unrolled group)
+#pragma unroll 1
       for (int q = 0; q < 4; ++q) {
+        // sign+mantissa bytes of this quarter: issued before its 16 symbols
+        uint4 smq = make_uint4(0, 0, 0, 0);
+        if (MODE == kFull) smq = __ldg(reinterpret_cast<const uint4*>(p.sm + e0) + q);
         // 16 symbols -> 4 words of exponent bytes (or 2 words of nibbles)
         uint32_t v[4] = {0, 0, 0, 0};
 #pragma unroll
@@ -212,7 +215,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_kernel(const DecodePara
           }
         }
         if (MODE == kFull) {
-          const uint4 s = smv[q];
+          const uint4 s = smq;
           uint32_t o[8];
           rebuild4(s.x, v[0], o[0], o[1]);
           rebuild4(s.y, v[1], o[2], o[3]);

@@ -237,15 +237,35 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   const int G = p.groups;
   const int warp_epi0 = kWarpRebuild0 + 4 * G;
 
+  const int mt_first = static_cast<int>((u0 / p.KB) / p.n_ntiles);
+  const int mt_last = static_cast<int>(((u1 - 1) / p.KB) / p.n_ntiles);
+  // pack records: this CTA's record offsets, loaded first of all (by the
+  // producer warp, while the MMA warp sets up barriers and tensor memory) --
+  // the first weight copy waits for them
+  uint32_t* soff = reinterpret_cast<uint32_t*>(smem + p.soff_off);
+  const int64_t pt_min = static_cast<int64_t>(mt_first) * p.KB;
   if (kPack && warp == kWarpProducer) {
-    // this CTA's record offsets: start pulling them into L2 while the CTA
-    // sets up (one 128-byte line per lane and step)
-    const int64_t pt0 = ((u0 / p.KB) / p.n_ntiles) * static_cast<int64_t>(p.KB);
     const int64_t n_tiles_total = static_cast<int64_t>((p.N + 127) / 128) * p.KB;
-    const int64_t cnt = p.n_soff < n_tiles_total + 1 - pt0 ? p.n_soff : n_tiles_total + 1 - pt0;
-    for (int64_t w = static_cast<int64_t>(lane) * 32; w < cnt; w += 32 * 32) prefetch_l2(p.pack_off + pt0 + w);
+    const int64_t want = static_cast<int64_t>(mt_last - mt_first + 1) * p.KB + 1;
+    const int64_t cnt = want < p.n_soff ? want : p.n_soff;
+    // all loads of a 256-word chunk are in flight before the first store:
+    // one memory round trip per chunk instead of one per word and lane
+    for (int64_t w0 = 0; w0 < cnt; w0 += 256) {
+      uint32_t v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t w = w0 + j * 32 + lane;
+        v[j] = (w < cnt && pt_min + w <= n_tiles_total) ? __ldg(p.pack_off + pt_min + w) : 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t w = w0 + j * 32 + lane;
+        if (w < cnt) soff[w] = v[j];
+      }
+    }
+    __syncwarp();
   }
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 32 * kWarpMma) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&bars->full[s], 1);
       mbar_init(&bars->rebuilt[s], 4);
@@ -283,8 +303,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 
   if (warp == kWarpProducer) {
     // ------------------------------ producer --------------------------------
-    const int mt_first = static_cast<int>((u0 / p.KB) / p.n_ntiles);
-    const int mt_last = static_cast<int>(((u1 - 1) / p.KB) / p.n_ntiles);
     uint32_t* meta = reinterpret_cast<uint32_t*>(smem + p.meta_off);
     int meta_issued[2] = {0, 0};
     // per-m-tile verbatim flags and prefix counts for its 128 rows
@@ -313,30 +331,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     if (kIdx4) {
       issue_meta(mt_first, 0);
       if (mt_first + 1 <= mt_last) issue_meta(mt_first + 1, 1);
-    }
-    // pack records: offsets of every record this CTA can touch
-    uint32_t* soff = reinterpret_cast<uint32_t*>(smem + p.soff_off);
-    const int64_t pt_min = static_cast<int64_t>(mt_first) * p.KB;
-    if (kPack) {
-      const int64_t n_tiles_total = static_cast<int64_t>((p.N + 127) / 128) * p.KB;
-      const int64_t want = static_cast<int64_t>(mt_last - mt_first + 1) * p.KB + 1;
-      const int64_t cnt = want < p.n_soff ? want : p.n_soff;
-      // all loads of a 256-word chunk are in flight before the first store:
-      // one memory round trip per chunk instead of one per word and lane
-      for (int64_t w0 = 0; w0 < cnt; w0 += 256) {
-        uint32_t v[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int64_t w = w0 + j * 32 + lane;
-          v[j] = (w < cnt && pt_min + w <= n_tiles_total) ? __ldg(p.pack_off + pt_min + w) : 0u;
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int64_t w = w0 + j * 32 + lane;
-          if (w < cnt) soff[w] = v[j];
-        }
-      }
-      __syncwarp();
     }
     int cur_mt = -1;
     int64_t i = 0;
