@@ -39,9 +39,9 @@ HBM_FALLBACK_GBS = 6650.0
 # of the direct-palette GEMM kernel (the 14336x4096 gate projection at batch 8,
 # ncu --set full; profiles/gemm_direct_palette_14336x4096_b8.md), valid only
 # for the kernel sources it was taken on: reported as null once they change.
-NCU_TRAFFIC = {"bytes_per_launch": 94127104,
+NCU_TRAFFIC = {"bytes_per_launch": 93671936,
                "launch": "gate projection 14336x4096, batch 8",
-               "sources_sha256": "7457d830303467e8f1c709171d999d83effeb4fc0f190b0ce26a34f781f37ddb"}
+               "sources_sha256": "a52c572650b091b2a70c886085391fe725eba75b2b22ace8bd335a18d8ef1d1f"}
 GEMM_SOURCES = ["mlp_huffman_coded_b200/csrc/uw_gemm.cu", "mlp_huffman_coded_b200/csrc/uw_device.cuh",
                 "mlp_huffman_coded_b200/csrc/uw_internal.h"]
 
