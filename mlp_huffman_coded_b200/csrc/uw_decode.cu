@@ -9,12 +9,14 @@
 //
 // Parallel structure: the stream is cut into chunks of `chunk_groups`
 // 64-element groups, each with its own start bit, so one thread decodes one
-// chunk from start to end.  The canonical code is decoded through an
-// 11-bit lookup table in shared memory (symbol, length, exponent per entry);
+// chunk from start to end.  The canonical code is decoded through a table in
+// shared memory indexed by the next 11 bits, which yields every whole code in
+// them at once (up to 4 symbols: their outputs and cumulative lengths);
 // longer codes (rare: the tail of the exponent distribution) fall back to the
-// canonical first-code comparison.  Each group's output (64 elements) goes
-// straight from registers to global memory in 16-byte stores; sign+mantissa
-// bytes are fetched with 16-byte loads issued before the group is decoded.
+// canonical first-code comparison.  Each 16-symbol quarter of a group is
+// gathered in 64-bit registers and goes to global memory in one store;
+// sign+mantissa bytes are fetched with a 16-byte load issued before the
+// quarter is decoded.
 // Verbatim groups (flag bit set) are copied from the verbatim store instead
 // and consume no stream bits.
 #include <cuda_runtime.h>
@@ -54,6 +56,12 @@ struct DecodeParams {
 
 struct DecodeTables {
   uint16_t lut[kLutSize];  // sym | len << 4 | exp << 8; len 0 = not in table
+  // Several symbols per lookup: for each 11-bit prefix, the whole codes it
+  // holds (at most 4): bits 0..31 their outputs (exponent bytes, or palette
+  // nibbles for the transcode), bits 32..47 the cumulative code lengths
+  // after 1..4 symbols (4 bits each), bits 48..50 the count (0: the first
+  // code is longer than the table).
+  uint64_t multi[kLutSize];
   uint32_t first[17];      // first canonical code of each length
   uint32_t count[17];      // codes of each length
   uint32_t offset[17];     // index of the first symbol of each length
@@ -61,7 +69,7 @@ struct DecodeTables {
   uint8_t palette[16];
 };
 
-__device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables& t) {
+__device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables& t, bool mode_idx4) {
   if (threadIdx.x == 0) {
     for (int l = 0; l <= 16; ++l) t.count[l] = 0;
     for (int i = 0; i < 16; ++i)
@@ -95,13 +103,30 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables
     t.lut[v] = ent;
   }
   __syncthreads();
+  // chain single-symbol lookups inside the 11-bit prefix: a code shorter than
+  // the bits left is decoded correctly whatever the zero padding (prefix-free)
+  for (int v = threadIdx.x; v < kLutSize; v += blockDim.x) {
+    uint64_t payload = 0, cum = 0;
+    int used = 0, n = 0;
+    while (n < 4 && used < kLutBits) {
+      const uint32_t e = t.lut[(static_cast<uint32_t>(v) << used) & (kLutSize - 1)];
+      const int l = (e >> 4) & 15;
+      if (l == 0 || l > kLutBits - used) break;
+      const uint64_t out = mode_idx4 ? (e & 15u) : (e >> 8);
+      payload |= out << (mode_idx4 ? 4 * n : 8 * n);
+      used += l;
+      cum |= static_cast<uint64_t>(used) << (4 * n);
+      ++n;
+    }
+    t.multi[v] = payload | (cum << 32) | (static_cast<uint64_t>(n) << 48);
+  }
+  __syncthreads();
 }
 
-// Codes longer than the table (rare: the tail of the exponent distribution)
-// by canonical first-code comparison.  Out of line: the symbol loop inlines
-// the table path dozens of times and this loop would bloat every copy.
-// On an invalid code records UW_ERR_CORRUPT and returns a length-1 entry so
-// decoding stays bounded.
+// A code longer than the table (rare: the tail of the exponent distribution)
+// by canonical first-code comparison, as a single-symbol entry (sym | len << 4
+// | exponent << 8).  On an invalid code records UW_ERR_CORRUPT and returns a
+// length-1 entry so decoding stays bounded.
 __device__ __forceinline__ uint32_t decode_long(const DecodeTables& t, int max_len, uint32_t* status,
                                              uint64_t win) {
   for (int l = kLutBits + 1; l <= max_len; ++l) {
@@ -116,18 +141,10 @@ __device__ __forceinline__ uint32_t decode_long(const DecodeTables& t, int max_l
   return 1u << 4;
 }
 
-// One canonical symbol from the top of a left-aligned 64-bit window, as a
-// table entry (sym | len << 4 | exponent << 8).
-__device__ __forceinline__ uint32_t decode_one(const DecodeTables& t, const DecodeParams& p,
-                                               uint64_t win) {
-  const uint32_t ent = t.lut[static_cast<uint32_t>(win >> (64 - kLutBits))];
-  return ((ent >> 4) & 15) != 0 ? ent : decode_long(t, p.max_len, p.status, win);
-}
-
 template <int MODE>
 __global__ void __launch_bounds__(kDecodeThreads, 7) decode_kernel(const DecodeParams p) {
   __shared__ DecodeTables t;
-  build_tables(p, t);
+  build_tables(p, t, MODE == kIdx4);
   const int64_t last_word = p.stream_words - 1;
   for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < p.n_chunks;
        c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -191,29 +208,48 @@ __global__ void __launch_bounds__(kDecodeThreads, 7) decode_kernel(const DecodeP
         // sign+mantissa bytes of this quarter: issued before its 16 symbols
         uint4 smq = make_uint4(0, 0, 0, 0);
         if (MODE == kFull) smq = __ldg(reinterpret_cast<const uint4*>(p.sm + e0) + q);
-        // 16 symbols -> 4 words of exponent bytes (or 2 words of nibbles)
-        uint32_t v[4] = {0, 0, 0, 0};
-#pragma unroll
-        for (int e = 0; e < 16; e += 2) {
+        // 16 symbols -> 16 exponent bytes (a0 | a1 << 64) or 16 nibbles (a0),
+        // several symbols per table lookup
+        uint64_t a0 = 0, a1 = 0;
+        int pos = 0;
+        while (pos < 16) {
           if (nb < 32) {
             win |= static_cast<uint64_t>(__ldg(p.stream + min(wi, last_word))) << (32 - nb);
             ++wi;
             nb += 32;
           }
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t ent = decode_one(t, p, win);
-            const uint32_t len = (ent >> 4) & 15;
-            win <<= len;
-            nb -= static_cast<int>(len);
-            consumed += len;
-            const int idx = e + h;
-            if (MODE == kIdx4)
-              v[idx >> 3] |= (ent & 15u) << (4 * (idx & 7));
-            else
-              v[idx >> 2] |= (ent >> 8) << (8 * (idx & 3));
+          const uint64_t ent = t.multi[static_cast<uint32_t>(win >> (64 - kLutBits))];
+          const int cnt = static_cast<int>((ent >> 48) & 7);
+          int k, len;
+          uint64_t pay;
+          if (cnt == 0) {  // a code longer than the table
+            const uint32_t e = decode_long(t, p.max_len, p.status, win);
+            k = 1;
+            len = static_cast<int>((e >> 4) & 15);
+            pay = MODE == kIdx4 ? (e & 15u) : (e >> 8);
+          } else {
+            k = min(cnt, 16 - pos);
+            len = static_cast<int>((ent >> (32 + 4 * (k - 1))) & 15);
+            pay = ent & ((MODE == kIdx4 ? (1ull << (4 * k)) : (1ull << (8 * k))) - 1);
           }
+          if (MODE == kIdx4) {
+            a0 |= pay << (4 * pos);
+          } else {
+            const int bp = 8 * pos;
+            if (pos < 8) {
+              a0 |= pay << bp;
+              if (pos + k > 8) a1 |= pay >> (64 - bp);
+            } else {
+              a1 |= pay << (bp - 64);
+            }
+          }
+          win <<= len;
+          nb -= len;
+          consumed += static_cast<uint32_t>(len);
+          pos += k;
         }
+        const uint32_t v[4] = {static_cast<uint32_t>(a0), static_cast<uint32_t>(a0 >> 32), static_cast<uint32_t>(a1),
+                               static_cast<uint32_t>(a1 >> 32)};
         if (MODE == kFull) {
           const uint4 s = smq;
           uint32_t o[8];
