@@ -41,7 +41,7 @@ HBM_FALLBACK_GBS = 6650.0
 # for the kernel sources it was taken on: reported as null once they change.
 NCU_TRAFFIC = {"bytes_per_launch": 93671936,
                "launch": "gate projection 14336x4096, batch 8",
-               "sources_sha256": "a52c572650b091b2a70c886085391fe725eba75b2b22ace8bd335a18d8ef1d1f"}
+               "sources_sha256": "0a01a6076c0595007d75291e16f7b5ed17cf3a882a8664fc575684b48851996e"}
 GEMM_SOURCES = ["mlp_huffman_coded_b200/csrc/uw_gemm.cu", "mlp_huffman_coded_b200/csrc/uw_device.cuh",
                 "mlp_huffman_coded_b200/csrc/uw_internal.h"]
 

@@ -128,7 +128,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* 
   return __all_sync(0xFFFFFFFFu, ok);
 }
 
-__device__ __forceinline__ bool group_and(bool v) {  // warps 6..9 (named barrier 1)
+__device__ __forceinline__ bool group_and(bool v) {  // the 4 epilogue warps (named barrier 1)
   uint32_t out;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
@@ -476,10 +476,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     }
   } else if (warp == kWarpMma) {
     // ----------------------------- MMA issuer -------------------------------
-    // One thread issues every MMA.  An M=128, K=16 tcgen05.mma occupies the
-    // tensor pipe for a fixed ~100+ cycles even at N=16, so at decode-sized
-    // batches this thread sets the pace: its loop carries all indices
-    // incrementally and does nothing but wait, issue and commit.
+    // One thread issues every MMA (one thread issues an M=128, K=16
+    // tcgen05.mma about every 50 cycles at N <= 64, so a 64-column stage costs
+    // ~0.1 us of issue plus its two barrier waits and commit).  The loop
+    // carries all indices incrementally and does nothing but wait, issue and
+    // commit.
     if (lane == 0) {
       int s = 0;
       uint32_t k = 0;
