@@ -542,6 +542,85 @@ def run_sweep_case(args, local):
     return 0
 
 
+def run_stack_case(args):
+    """Compressed size of the 32-layer MLP stack (96 matrices, per-layer sigma
+    uniform in [0.01, 0.05], 1e-3 outliers x100): host encoder only, no GPU."""
+    from mlp_huffman_coded_b200 import synth, uw
+    n_layers = args.layers
+    tot = dict(bf16=0, huffman=0, pack=0, verbatim=0, groups=0, bits=0, coded=0)
+    for layer in range(n_layers):
+        for name, w in zip(("gate", "up", "down"), synth.stack_layer(layer)):
+            e = uw.encode(w)
+            _, pack = e.pack_offsets()
+            nv, ng = int(e.layout.n_verbatim), int(e.layout.n_groups)
+            bits = int(e.chunk_bit_off[-1])
+            tot["bf16"] += w.nbytes
+            tot["huffman"] += e.compressed_bytes("huffman")
+            tot["pack"] += pack
+            tot["verbatim"] += nv
+            tot["groups"] += ng
+            tot["bits"] += bits
+            tot["coded"] += (ng - nv) * 64
+            print(json.dumps({"case": "stack", "layer": layer, "matrix": name,
+                              "sigma": round(float(synth.stack_sigmas()[layer]), 5), "bf16_bytes": w.nbytes,
+                              "huffman_ratio": e.compressed_bytes("huffman") / w.nbytes,
+                              "pack_ratio": pack / w.nbytes, "verbatim_frac": nv / ng,
+                              "mean_code_bits": bits / max(1, (ng - nv) * 64)}), flush=True)
+    print(json.dumps({"case": "stack", "layers": n_layers, "matrices": 3 * n_layers,
+                      "bf16_gb": tot["bf16"] / 1e9, "huffman_gb": tot["huffman"] / 1e9,
+                      "huffman_ratio": tot["huffman"] / tot["bf16"], "pack_gb": tot["pack"] / 1e9,
+                      "pack_ratio": tot["pack"] / tot["bf16"], "verbatim_frac": tot["verbatim"] / tot["groups"],
+                      "mean_code_bits": tot["bits"] / max(1, tot["coded"])}), flush=True)
+    return 0
+
+
+def run_stack_time_case(args, local):
+    """Per-decode-step MLP time of the 32-layer stack at batch 1 and 64 with
+    the autotuned pipeline per matrix, measured on the first `--layers`
+    layers (a sample: loading all 96 matrices would take minutes of host
+    encoding) and scaled to 32 layers -- labelled as such."""
+    import torch
+    from mlp_huffman_coded_b200 import synth, uw
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    batches = [1, 64]
+    flush = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+    ws0 = uw.Workspace(256, device=dev)
+    per_layer = {b: [] for b in batches}
+    for layer in range(args.layers):
+        dms = [uw.DeviceMatrix(uw.encode(w), device=dev).prepare_direct_palette(ws0) for w in synth.stack_layer(layer)]
+        ws0.check("prepare")
+        choices = []
+        for dm in dms:
+            K = int(dm.mat.L.cols)
+            wsa = uw.Workspace(max(uw.workspace_bytes(dm, p, max(batches)) for p in range(4)), device=dev)
+            xa = torch.from_numpy(synth.activations(max(batches), K, 3).view(np.int16)).to(dev)
+            ya = torch.empty(max(batches), int(dm.mat.L.rows), dtype=torch.int16, device=dev)
+            ch, _ = uw.autotune(dm, batches, 5, xa, ya, wsa, flush=flush)
+            wsa.check("autotune")
+            choices.append(ch)
+            del wsa
+        for bi, B in enumerate(batches):
+            pipes = [c[bi] for c in choices]
+            ws = uw.Workspace(uw.mlp_workspace_bytes(*dms, pipes, B), device=dev)
+            x = torch.from_numpy(synth.activations(B, D_MODEL, 3).view(np.int16)).to(dev)
+            y = torch.empty(B, D_MODEL, dtype=torch.int16, device=dev)
+            med, mn = _timed(lambda: uw.mlp_block(*dms, pipes, x, y, ws), flush, args.steps, args.warmup, dev)
+            ws.check("stack block")
+            per_layer[B].append(med)
+            print(json.dumps({"case": "stack-time", "layer": layer, "batch": B,
+                              "pipelines": [uw.PIPE_NAMES[p] for p in pipes], "block_us": med}), flush=True)
+        del dms
+        torch.cuda.empty_cache()
+    for B in batches:
+        mean = float(np.mean(per_layer[B]))
+        print(json.dumps({"case": "stack-time", "batch": B, "layers_measured": args.layers,
+                          "mean_block_us": mean, "step_32_layers_ms_extrapolated": 32 * mean / 1e3,
+                          "note": "L2 flushed before each block; the 32-layer figure is 32 x the measured mean"}),
+              flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -552,16 +631,22 @@ def main(argv=None):
     ap.add_argument("--impl", default="uw", choices=["uw", "reference"])
     ap.add_argument("--ref-fraction", type=float, default=1 / 16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--case", default="block", choices=["block", "gemm", "decode", "sweep"],
+    ap.add_argument("--layers", type=int, default=32, help="stack / stack-time cases: layers to use")
+    ap.add_argument("--case", default="block", choices=["block", "gemm", "decode", "sweep", "stack", "stack-time"],
                     help="gemm: one 14336x4096 matrix through --pipeline (profiling unit); decode: the three "
-                         "decoders on it; sweep: pipelines x batch 1..512 x block matrices + autotune")
+                         "decoders on it; sweep: pipelines x batch 1..512 x block matrices + autotune; "
+                         "stack: compressed size of the 32-layer stack (host only); stack-time: block time "
+                         "of its first --layers layers at batch 1 and 64")
     ap.add_argument("--pipeline", default="direct", choices=["full", "exponent", "transcode", "direct", "bf16"])
     ap.add_argument("--no-flush", action="store_true", help="gemm case: leave L2 warm between calls")
     args = ap.parse_args(argv)
     if args.steps is None:
-        args.steps = 20 if args.impl == "reference" else {"gemm": 100, "decode": 20, "sweep": 10}.get(args.case, 3000)
+        args.steps = 20 if args.impl == "reference" else {"gemm": 100, "decode": 20, "sweep": 10,
+                                                         "stack-time": 20}.get(args.case, 3000)
     if args.warmup is None:
-        args.warmup = 3 if args.impl == "reference" or args.case in ("sweep", "decode") else 20
+        args.warmup = 3 if args.impl == "reference" or args.case in ("sweep", "decode", "stack-time") else 20
+    if args.case == "stack":
+        return run_stack_case(args)
     world, rank, local = dist_init()
     try:
         if args.impl == "reference":
@@ -572,6 +657,8 @@ def main(argv=None):
             return run_decode_case(args, local)
         if args.case == "sweep":
             return run_sweep_case(args, local)
+        if args.case == "stack-time":
+            return run_stack_time_case(args, local)
         return run_gpu(args, world, rank, local)
     finally:
         if world > 1:

@@ -22,6 +22,7 @@ __all__ = [
     "small_integer_matrix",
     "WORKLOADS",
     "stack_sigmas",
+    "stack_layer",
 ]
 
 
@@ -106,6 +107,17 @@ WORKLOADS = {
     "mlp_block_4096_14336": dict(d_model=4096, ffn=14336, sigma=0.02, outlier_rate=1e-4,
                                  outlier_scale=100.0, seed=2),
 }
+
+
+def stack_layer(layer: int, n_layers: int = 32, d_model: int = 4096, ffn: int = 14336,
+                outlier_rate: float = 1e-3, outlier_scale: float = 100.0):
+    """Layer `layer` of the 32-layer MLP stack: gate [ffn, d], up [ffn, d],
+    down [d, ffn] with the layer's sigma and seeds 2000 + 3*layer + j."""
+    sigma = float(stack_sigmas(n_layers)[layer])
+    seed = 2000 + 3 * layer
+    return (weight_matrix(ffn, d_model, sigma, outlier_rate, outlier_scale, seed),
+            weight_matrix(ffn, d_model, sigma, outlier_rate, outlier_scale, seed + 1),
+            weight_matrix(d_model, ffn, sigma, outlier_rate, outlier_scale, seed + 2))
 
 
 def mlp_block(d_model: int = 4096, ffn: int = 14336, sigma: float = 0.02,
