@@ -78,6 +78,12 @@
  *     launched.  Problems the GPU finds (a corrupt stream, a wait that ran
  *     out of time) are recorded in the workspace's status word and read back
  *     with uw_workspace_status().
+ *   - GEMM kernels are launched with programmatic dependent launch: one may
+ *     start streaming its (constant) weights while the previous kernel on
+ *     the same stream is still running, and waits for that kernel to
+ *     complete before it reads x or the SwiGLU gate, or writes y or the
+ *     workspace.  Ordering through events, copies or other streams is the
+ *     usual full ordering.
  *   - Host calls (uw_build_palette_codebook, uw_encode, uw_validate) are
  *     synchronous and thread-safe.
  *   - Device pointers must be 16-byte aligned; violations give
