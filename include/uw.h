@@ -82,8 +82,14 @@
  *     start streaming its (constant) weights while the previous kernel on
  *     the same stream is still running, and waits for that kernel to
  *     complete before it reads x or the SwiGLU gate, or writes y or the
- *     workspace.  Ordering through events, copies or other streams is the
- *     usual full ordering.
+ *     workspace.  A GEMM that follows its own decode kernel (full,
+ *     exponent-only and transcode pipelines) is launched plainly, and
+ *     uw_pack_direct_palette ends with a plainly launched empty kernel, so a
+ *     GEMM never reads weights before the kernel that wrote them is done.
+ *     Weights written by a caller's kernel must likewise be followed by a
+ *     plain stream operation (another kernel, an event, a copy) before the
+ *     GEMM.  Ordering through events, copies or other streams is the usual
+ *     full ordering.
  *   - Host calls (uw_build_palette_codebook, uw_encode, uw_validate) are
  *     synchronous and thread-safe.
  *   - Device pointers must be 16-byte aligned; violations give

@@ -893,7 +893,7 @@ bool make_layout(int loader, const GemmPlan& plan, int wpr, bool tma_out, bool g
 
 template <int L>
 uw_status launch_kernel(const CUtensorMap& x, const CUtensorMap& wa, const CUtensorMap& wb, const CUtensorMap& y,
-                        const CUtensorMap& g, const KParams& kp, size_t smem, cudaStream_t s) {
+                        const CUtensorMap& g, const KParams& kp, size_t smem, cudaStream_t s, bool overlap) {
   static std::once_flag once[64];
   static cudaError_t attr_err[64];
   int dev = 0;
@@ -914,7 +914,7 @@ uw_status launch_kernel(const CUtensorMap& x, const CUtensorMap& wa, const CUten
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].val.programmaticStreamSerializationAllowed = overlap ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const cudaError_t launch_err = cudaLaunchKernelEx(&cfg, gemm_kernel<L>, x, wa, wb, y, g, kp);
@@ -1072,12 +1072,12 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.tma_out = tma_out ? 1 : 0;
 
   switch (kl) {
-    case kBF16: return launch_kernel<kBF16>(tx, twa, twb, ty, tg, kp, lay.smem, s);
-    case kEXP8: return launch_kernel<kEXP8>(tx, twa, twb, ty, tg, kp, lay.smem, s);
-    case kIDX4U: return launch_kernel<kIDX4U>(tx, twa, twb, ty, tg, kp, lay.smem, s);
-    case kIDX4M: return launch_kernel<kIDX4M>(tx, twa, twb, ty, tg, kp, lay.smem, s);
-    case kPACKU: return launch_kernel<kPACKU>(tx, twa, twb, ty, tg, kp, lay.smem, s);
-    default: return launch_kernel<kPACKM>(tx, twa, twb, ty, tg, kp, lay.smem, s);
+    case kBF16: return launch_kernel<kBF16>(tx, twa, twb, ty, tg, kp, lay.smem, s, a.overlap_previous);
+    case kEXP8: return launch_kernel<kEXP8>(tx, twa, twb, ty, tg, kp, lay.smem, s, a.overlap_previous);
+    case kIDX4U: return launch_kernel<kIDX4U>(tx, twa, twb, ty, tg, kp, lay.smem, s, a.overlap_previous);
+    case kIDX4M: return launch_kernel<kIDX4M>(tx, twa, twb, ty, tg, kp, lay.smem, s, a.overlap_previous);
+    case kPACKU: return launch_kernel<kPACKU>(tx, twa, twb, ty, tg, kp, lay.smem, s, a.overlap_previous);
+    default: return launch_kernel<kPACKM>(tx, twa, twb, ty, tg, kp, lay.smem, s, a.overlap_previous);
   }
 }
 
@@ -1128,11 +1128,13 @@ uw_status run_pipeline(const uw_matrix* m, int pipeline, const uint16_t* x, int3
     case UW_PIPE_FULL:
       if ((st = launch_decode(m, 0, scratch, status, s)) != UW_OK) return st;
       a.loader = kLoaderBF16;
+      a.overlap_previous = false;  // its weights are the decode kernel's output
       a.wbf16 = static_cast<const uint16_t*>(scratch);
       break;
     case UW_PIPE_EXPONENT:
       if ((st = launch_decode(m, 1, scratch, status, s)) != UW_OK) return st;
       a.loader = kLoaderEXP8;
+      a.overlap_previous = false;
       a.sm = m->sm;
       a.aux = static_cast<const uint8_t*>(scratch);
       break;
@@ -1151,6 +1153,7 @@ uw_status run_pipeline(const uw_matrix* m, int pipeline, const uint16_t* x, int3
       if ((st = launch_decode(m, 2, scratch, status, s)) != UW_OK) return st;
       const uint8_t* idx4 = static_cast<const uint8_t*>(scratch);
       a.loader = kLoaderIDX4;
+      a.overlap_previous = false;
       a.sm = m->sm;
       a.aux = idx4;
       a.vflags = m->vflags;

@@ -83,6 +83,10 @@ struct GemmArgs {
   void* ws = nullptr;
   size_t ws_bytes = 0;
   int force_mixed_palette = 0;        // testing: use the general lookup
+  // Launch with programmatic dependent launch (the kernel streams its weights
+  // before waiting for the previous kernel on the stream).  Off when that
+  // previous kernel wrote the weights (a decode kernel of the same call).
+  bool overlap_previous = true;
 };
 uw_status launch_gemm(const GemmArgs& a, cudaStream_t s);
 uw_status launch_swiglu(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t n, cudaStream_t s);

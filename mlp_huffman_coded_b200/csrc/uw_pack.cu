@@ -83,6 +83,10 @@ __global__ void __launch_bounds__(128) pack_kernel(const PackParams p) {
   }
 }
 
+// Does nothing: launched plainly after the pack kernel as a stream-ordering
+// point (see uw_pack_direct_palette).
+__global__ void ordering_kernel() {}
+
 }  // namespace
 }  // namespace uw
 
@@ -110,6 +114,13 @@ extern "C" uw_status uw_pack_direct_palette(const uw_matrix* m, const uint32_t* 
   const int64_t n_tiles = ((m->L.rows + 127) / 128) * p.KB;
   if (n_tiles > 0x7FFFFFFF) return UW_ERR_UNSUPPORTED_SHAPE;
   pack_kernel<<<static_cast<unsigned>(n_tiles), 128, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  note_launch();
+  if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return cuda_status(e);
+  // GEMM kernels stream their weights before waiting on the kernel ahead of
+  // them (programmatic dependent launch).  A plainly launched empty kernel
+  // after the pack starts only once the pack is complete and visible, so a
+  // GEMM queued next can never read a record early.
+  ordering_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
   note_launch();
   return cuda_status(cudaGetLastError());
 }
