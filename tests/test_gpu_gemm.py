@@ -56,6 +56,15 @@ def test_ragged_shapes(rows, cols):
     _check_gemm(w, x)
 
 
+@pytest.mark.parametrize("rows,cols,B", [(203, 512, 1), (203, 512, 40), (1001, 192, 8), (77, 64, 300)])
+def test_rows_not_multiple_of_8_use_per_element_stores(rows, cols, B):
+    # output rows of N*2 bytes are not 16-byte multiples: the epilogue cannot
+    # use TMA tensor stores and writes element by element
+    w = synth.weight_matrix(rows, cols, 0.02, 2e-3, 100.0, rows * 7 + cols)
+    x = synth.activations(B, cols, 9)
+    _check_gemm(w, x)
+
+
 def test_one_hot_input_selects_a_column_exactly():
     w = synth.weight_matrix(384, 1024, 0.02, 2e-3, 100.0, 40)
     dm = device_matrix(w)
