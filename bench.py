@@ -144,24 +144,26 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(world, v: float) -> float:
+def _reduce_over_ranks(world, v: float, op) -> float:
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    # NCCL reduces device tensors; gloo (CPU tests) host tensors
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
     return float(t.item())
+
+
+def max_over_ranks(world, v: float) -> float:
+    import torch.distributed as dist
+    return _reduce_over_ranks(world, v, dist.ReduceOp.MAX)
 
 
 def sum_over_ranks(world, v: float) -> float:
-    if world == 1:
-        return v
-    import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _reduce_over_ranks(world, v, dist.ReduceOp.SUM)
 
 
 # ---------------------------------------------------------------------------
