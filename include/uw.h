@@ -245,6 +245,20 @@ UW_API uw_status uw_workspace_init(void* workspace, size_t workspace_bytes, void
  * first problem any kernel recorded since the last read) and clear it. */
 UW_API uw_status uw_workspace_status(void* workspace, void* stream);
 
+/* Self-test of the bounded waits (no counterpart on the page: a robustness
+ * check of this library).  Every wait in these kernels -- on an mbarrier
+ * phase or on another CTA's counter -- gives up after a time limit, records
+ * UW_ERR_TIMEOUT in the workspace status word and lets the kernel return.
+ * This launches one warp that waits on a phase nothing completes and then on
+ * a counter nothing increments, each for `limit_us` microseconds (1 ..
+ * 1000000): afterwards uw_workspace_status() returns UW_ERR_TIMEOUT and the
+ * CUDA context stays usable.  Uses header bytes [64, 80) of the workspace
+ * (words 0 and 1 end as 0 when both waits gave up).  Errors:
+ * UW_ERR_INVALID_ARG (NULL / misaligned / smaller than 256 bytes / limit out
+ * of range), UW_ERR_NO_DEVICE, UW_ERR_CUDA. */
+UW_API uw_status uw_selftest_bounded_wait(void* workspace, size_t workspace_bytes, uint32_t limit_us,
+                                          void* stream);
+
 /* ---------------------------------------------------------------------------
  * Preprocessing kernels (section "Four ways to use compressed weights")
  * ------------------------------------------------------------------------- */

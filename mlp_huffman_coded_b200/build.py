@@ -24,7 +24,7 @@ LIB = os.path.join(PKG, "libuw.so")
 BUILD_DIR = os.path.join(PKG, "_build")
 
 SOURCES = ["uw_host.cpp", "uw_runtime.cu", "uw_decode.cu", "uw_pack.cu", "uw_gemm.cu", "uw_autotune.cu",
-           "uw_noalloc.cu"]
+           "uw_noalloc.cu", "uw_selftest.cu"]
 HEADERS = ["uw_device.cuh", "uw_internal.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -66,23 +66,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Bounded wait for the phase with the given parity to complete.  Returns
-// false (after recording UW_ERR_TIMEOUT and raising *abort) when the limit
+// false (after recording UW_ERR_TIMEOUT and raising *abort) when `limit_ns`
 // passes or another thread has already raised *abort.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
-                                          uint32_t* status) {
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
+                                              uint32_t* status, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63) == 63) {
       if (abort && *abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         record_status(status, UW_ERR_TIMEOUT);
         if (abort) *abort = 1;
         return false;
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile uint32_t* abort,
+                                          uint32_t* status) {
+  return mbar_wait_for(bar, parity, abort, status, kWaitLimitNs);
 }
 
 // ---------------------------------------------------------------------------
@@ -146,6 +151,27 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+// Bounded spin until *counter >= want (another CTA's release add): false
+// (after recording UW_ERR_TIMEOUT and raising *abort) when `limit_ns` passes
+// or another thread has already raised *abort.
+__device__ __forceinline__ bool wait_count_at_least(const uint32_t* counter, uint32_t want,
+                                                    volatile uint32_t* abort, uint32_t* status,
+                                                    uint64_t limit_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0; ld_acquire_gpu(counter) < want; ++it) {
+    if ((it & 15) == 15) {
+      if (abort && *abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        record_status(status, UW_ERR_TIMEOUT);
+        if (abort) *abort = 1;
+        return false;
+      }
+    }
+    __nanosleep(100);
+  }
+  return true;
+}
+
 // Publish: every write this thread has observed (including other threads'
 // writes ordered before it by a CTA barrier) becomes visible before the add.
 __device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {

@@ -681,21 +681,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       bool staged = false;
       if (reducer) {
         bool got = true;
-        if (elected) {
-          const uint64_t w0 = globaltimer_ns();
-          for (uint32_t it = 0; ld_acquire_gpu(p.counters + t) < static_cast<uint32_t>(ncontrib - 1); ++it) {
-            if ((it & 15) == 15) {
-              if (bars->abort) { got = false; break; }
-              if (globaltimer_ns() - w0 > kWaitLimitNs) {
-                record_status(p.status, UW_ERR_TIMEOUT);
-                bars->abort = 1;
-                got = false;
-                break;
-              }
-            }
-            __nanosleep(100);
-          }
-        }
+        if (elected)
+          got = wait_count_at_least(p.counters + t, static_cast<uint32_t>(ncontrib - 1), &bars->abort, p.status,
+                                    kWaitLimitNs);
         if (!group_and(got)) break;  // also orders the partial loads after the acquire
         // on the CTA's last segment every stage has been consumed: copy the
         // other partials of this thread's row into the stage buffers at once

@@ -64,6 +64,7 @@ _SIGS = {
                             _P, _P, _P, _P, _P, _P]),
     "uw_validate": (C.c_int, [C.POINTER(Matrix)]),
     "uw_direct_pack_offsets": (C.c_int, [C.POINTER(Layout), _P, _P, C.POINTER(C.c_uint64)]),
+    "uw_selftest_bounded_wait": (C.c_int, [_P, C.c_size_t, C.c_uint32, _P]),
     "uw_pack_direct_palette": (C.c_int, [C.POINTER(Matrix), _P, _P, _P]),
     "uw_workspace_bytes": (C.c_size_t, [C.POINTER(Layout), C.c_int32, C.c_int32]),
     "uw_workspace_init": (C.c_int, [_P, C.c_size_t, _P]),
@@ -378,6 +379,13 @@ def autotune(dm: DeviceMatrix, batches, reps: int, x, y, ws: Workspace, flush=No
                              0 if flush is None else flush.numel() * flush.element_size(), ws.ptr, ws.nbytes,
                              choice, us, _stream(stream)), "uw_autotune")
     return list(choice), np.array(list(us), dtype=np.float64).reshape(n, 4)
+
+
+def selftest_bounded_wait(ws: Workspace, limit_us: int, stream=None):
+    """Launch the bounded-wait self-test (see uw.h); the status it leaves is
+    read with ws.status()."""
+    _check(lib().uw_selftest_bounded_wait(ws.ptr, ws.nbytes, int(limit_us), _stream(stream)),
+           "uw_selftest_bounded_wait")
 
 
 def launch_count() -> int:
