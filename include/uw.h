@@ -210,16 +210,19 @@ UW_API uw_status uw_encode(const uint16_t* w_host, int64_t rows, int64_t cols, c
                     uint32_t* chunk_bit_off, uint32_t* vflags, uint32_t* vprefix,
                     uint16_t* verbatim);
 
-/* Record offsets (16-byte units) of the direct-palette pack of a matrix,
- * computed from its HOST vflags: pack_off[t+1] - pack_off[t] =
+/* Record offsets (16-byte units) of the direct-palette pack of a matrix
+ * (section "How the reconstructive matmul works": what the producer stages
+ * per tile -- sign+mantissa bytes, palette indices, verbatim rows; the byte
+ * layout is this library's), computed from its HOST vflags: pack_off[t+1] - pack_off[t] =
  * (12416 + 128*min(verbatim rows of tile t, 32)) / 16.  pack_off_host holds
  * n_tiles+1 entries; *pack_bytes (may be NULL) receives the total size.
  * Errors: UW_ERR_INVALID_ARG, UW_ERR_UNSUPPORTED_SHAPE (pack above 64 GiB). */
 UW_API uw_status uw_direct_pack_offsets(const uw_layout* L, const uint32_t* vflags_host,
                                         uint32_t* pack_off_host, uint64_t* pack_bytes);
 
-/* Host-side consistency check of a compressed matrix whose pointers are
- * HOST copies: canonical codebook with Kraft sum <= 1, offsets monotone and
+/* Host-side consistency check (no counterpart on the page: it checks the
+ * format of section "How to compress model weights effectively") of a
+ * compressed matrix whose pointers are HOST copies: canonical codebook with Kraft sum <= 1, offsets monotone and
  * ending at total_bits, vprefix equal to the running popcount of vflags,
  * sizes consistent.  Run it before uploading data from an untrusted file.
  * Errors: UW_ERR_INVALID_ARG, UW_ERR_CORRUPT. */
@@ -229,20 +232,25 @@ UW_API uw_status uw_validate(const uw_matrix* host_mirror);
  * Workspace
  * ------------------------------------------------------------------------- */
 
-/* Bytes of device workspace a device call needs for this matrix, pipeline
- * and batch (batch 0 for the decode/transcode calls).  The workspace holds a
+/* Bytes of device workspace (library plumbing; no counterpart on the page)
+ * a device call needs for this matrix, pipeline and batch (batch 0 for the
+ * decode/transcode calls).  The workspace holds a
  * status word, split-K partial sums and tile counters, and for the FULL /
  * EXPONENT / TRANSCODE pipelines the intermediate decoded matrix.  Returns 0
  * for invalid arguments. */
 UW_API size_t uw_workspace_bytes(const uw_layout* L, int32_t pipeline, int32_t batch);
 
-/* Zero a workspace (stream-ordered).  A workspace must be zeroed once before
- * its first use; afterwards every call leaves its counters at zero again.
- * Calls that share one workspace must be ordered on one stream. */
+/* Zero a workspace (stream-ordered; library plumbing).  A workspace must be
+ * zeroed once before its first use; afterwards every call leaves its
+ * counters at zero again.  Calls that share one workspace must be ordered on
+ * one stream.  Errors: UW_ERR_INVALID_ARG (NULL, misaligned, < 256 bytes),
+ * UW_ERR_CUDA. */
 UW_API uw_status uw_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronize the stream, read the workspace's sticky status word (the
- * first problem any kernel recorded since the last read) and clear it. */
+ * first problem any kernel recorded since the last read) and clear it
+ * (library plumbing).  Returns that status (UW_OK when none), or
+ * UW_ERR_INVALID_ARG / UW_ERR_CUDA for the read itself. */
 UW_API uw_status uw_workspace_status(void* workspace, void* stream);
 
 /* Self-test of the bounded waits (no counterpart on the page: a robustness
@@ -263,33 +271,42 @@ UW_API uw_status uw_selftest_bounded_wait(void* workspace, size_t workspace_byte
  * Preprocessing kernels (section "Four ways to use compressed weights")
  * ------------------------------------------------------------------------- */
 
-/* Full Huffman decode: out_bf16[rows*cols] (device, row-major BF16 bits)
- * gets back every original word bit for bit, verbatim groups copied from the
- * verbatim store.  Reads sm + stream + offsets + flags + verbatim; writes
- * 2 bytes per element.  A chunk whose code lengths do not end exactly at
- * the next chunk's offset records UW_ERR_CORRUPT. */
+/* Full Huffman decode (section "Four ways to use compressed weights", full
+ * decode): out_bf16[rows*cols] (device, row-major BF16 bits) gets back every
+ * original word bit for bit, verbatim groups copied from the verbatim store.
+ * Reads sm + stream + offsets + flags + verbatim; writes 2 bytes per
+ * element.  Errors: UW_ERR_INVALID_ARG (NULL or misaligned pointers),
+ * UW_ERR_WORKSPACE_TOO_SMALL (< 256 bytes), UW_ERR_NO_DEVICE, UW_ERR_CUDA;
+ * on the device, a chunk whose code lengths do not end exactly at the next
+ * chunk's offset (or an invalid code) records UW_ERR_CORRUPT in the status
+ * word, and every read stays inside the stream. */
 UW_API uw_status uw_decode_full(const uw_matrix* m, uint16_t* out_bf16, void* workspace,
                          size_t workspace_bytes, void* stream);
 
-/* Exponent-only decode: out_exp8[rows*cols] (device) = exponent byte of every
- * element (verbatim groups from the verbatim store); half of the full
- * decode's write traffic.  The GEMM recombines it with the raw sm bytes. */
+/* Exponent-only decode (section "Four ways to use compressed weights"):
+ * out_exp8[rows*cols] (device) = exponent byte of every element (verbatim
+ * groups from the verbatim store); half of the full decode's write traffic.
+ * The GEMM recombines it with the raw sm bytes.  Errors as uw_decode_full. */
 UW_API uw_status uw_decode_exponent_only(const uw_matrix* m, uint8_t* out_exp8, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
-/* Palette transcode: out_idx4[rows*cols/2] (device) = 4-bit palette index per
- * element in the idx4 layout, 0 in verbatim groups; a quarter of the full
- * decode's write traffic.  Run once at load time this is the "direct
- * palette" preparation; run per call it is the "palette transcode"
- * pipeline. */
+/* Palette transcode (section "Four ways to use compressed weights"):
+ * out_idx4[rows*cols/2] (device) = 4-bit palette index per element in the
+ * idx4 layout, 0 in verbatim groups; a quarter of the full decode's write
+ * traffic.  Run once at load time this is the "direct palette"
+ * preparation; run per call it is the "palette transcode" pipeline.
+ * Errors as uw_decode_full. */
 UW_API uw_status uw_transcode_palette(const uw_matrix* m, uint8_t* out_idx4, void* workspace,
                                size_t workspace_bytes, void* stream);
 
-/* Load-time assembly of the direct-palette pack (layout above) from sm,
- * m->idx4 (must be set) and the verbatim store, so that the direct-palette
- * GEMM streams one contiguous record per tile.  pack_off: device copy of the
- * offsets from uw_direct_pack_offsets; out_pack: device buffer of
- * 16*pack_off[n_tiles] bytes. */
+/* Load-time assembly of the direct-palette pack (sections "Four ways to use
+ * compressed weights", direct palette, and "How the reconstructive matmul
+ * works"; layout above) from sm, m->idx4 (must be set) and the verbatim
+ * store, so that the direct-palette GEMM streams one contiguous record per
+ * tile.  pack_off: device copy of the offsets from uw_direct_pack_offsets;
+ * out_pack: device buffer of 16*pack_off[n_tiles] bytes, written by this
+ * call (the caller owns it).  Errors: UW_ERR_INVALID_ARG (NULL, misaligned,
+ * m->idx4 unset), UW_ERR_UNSUPPORTED_SHAPE, UW_ERR_NO_DEVICE, UW_ERR_CUDA. */
 UW_API uw_status uw_pack_direct_palette(const uw_matrix* m, const uint32_t* pack_off,
                                         uint8_t* out_pack, void* stream);
 
@@ -297,7 +314,10 @@ UW_API uw_status uw_pack_direct_palette(const uw_matrix* m, const uint32_t* pack
  * Reconstructive GEMM (section "How the reconstructive matmul works")
  * ------------------------------------------------------------------------- */
 
-/* y = x W^T with the direct-palette matrix: x is device BF16 [batch, cols]
+/* Direct-palette reconstructive GEMM (section "How the reconstructive matmul
+ * works"; the "direct palette" pipeline of section "Four ways to use
+ * compressed weights").
+ * y = x W^T with the direct-palette matrix: x is device BF16 [batch, cols]
  * row-major, y is device BF16 [batch, rows] row-major.  W is rebuilt tile by
  * tile on chip from the pack records (sm + 4-bit indices + verbatim rows,
  * chosen once per 64-element row) and fed to tcgen05 MMA with FP32
@@ -311,16 +331,19 @@ UW_API uw_status uw_gemm_direct_palette(const uw_matrix* m, const uint16_t* x, i
                                  uint16_t* y, void* workspace, size_t workspace_bytes,
                                  void* stream);
 
-/* y = x W^T through any pipeline, including its preprocessing kernel (whose
- * output lives in the workspace).  UW_PIPE_BF16 is not accepted here (see
- * uw_gemm_bf16). */
+/* y = x W^T through any of the four pipelines of section "Four ways to use
+ * compressed weights", including its preprocessing kernel (whose output
+ * lives in the workspace).  UW_PIPE_BF16 is not accepted here (see
+ * uw_gemm_bf16).  Errors as uw_gemm_direct_palette, plus UW_ERR_INVALID_ARG
+ * for an unknown pipeline or a DIRECT call without m->pack. */
 UW_API uw_status uw_gemm(const uw_matrix* m, int32_t pipeline, const uint16_t* x, int32_t batch,
                   uint16_t* y, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Same as uw_gemm_direct_palette, but always uses the general palette lookup
  * (the one for palettes whose used exponents differ in their top bit)
  * instead of the faster single-table lookup.  Results are identical; this
- * entry point exists so the general lookup can be tested on any matrix. */
+ * entry point (no counterpart on the page) exists so the general lookup can
+ * be tested on any matrix.  Errors as uw_gemm_direct_palette. */
 UW_API uw_status uw_gemm_direct_palette_general_lookup(const uw_matrix* m, const uint16_t* x,
                                                        int32_t batch, uint16_t* y, void* workspace,
                                                        size_t workspace_bytes, void* stream);
@@ -350,9 +373,10 @@ UW_API uw_status uw_gemm_direct_palette_general_lookup(const uw_matrix* m, const
 UW_API uw_status uw_gemm_direct_palette_noalloc(const uw_matrix* m, const uint16_t* x, int32_t batch,
                                                 uint16_t* y, void* stream);
 
-/* Uncompressed comparator: y = x W^T with W given as device BF16
- * [rows, cols]; the same GEMM kernel, loader reading BF16 tiles.  Workspace:
- * uw_workspace_bytes with UW_PIPE_BF16. */
+/* Uncompressed comparator (the page's BF16 baseline; the "full decode"
+ * pipeline's GEMM step): y = x W^T with W given as device BF16 [rows, cols];
+ * the same GEMM kernel, loader reading BF16 tiles.  Workspace:
+ * uw_workspace_bytes with UW_PIPE_BF16.  Errors as uw_gemm_direct_palette. */
 UW_API uw_status uw_gemm_bf16(const uint16_t* w, int64_t rows, int64_t cols, const uint16_t* x,
                        int32_t batch, uint16_t* y, void* workspace, size_t workspace_bytes,
                        void* stream);
@@ -362,14 +386,21 @@ UW_API uw_status uw_gemm_bf16(const uint16_t* w, int64_t rows, int64_t cols, con
  * ------------------------------------------------------------------------- */
 
 /* h = bf16(SiLU(g) * u) elementwise over n BF16 values (device), computed in
- * FP32: SiLU(v) = v / (1 + exp(-v)). */
+ * FP32: SiLU(v) = v / (1 + exp(-v)).  The glue of a SwiGLU MLP block (the
+ * page compresses its gate/up/down matrices; the block itself is not on the
+ * page).  Errors: UW_ERR_INVALID_ARG (NULL with n > 0, n < 0),
+ * UW_ERR_NO_DEVICE, UW_ERR_CUDA. */
 UW_API uw_status uw_swiglu(const uint16_t* g, const uint16_t* u, uint16_t* h, int64_t n, void* stream);
 
-/* One SwiGLU MLP block: y = W_down (SiLU(W_gate x) * (W_up x)).  gate, up:
+/* One SwiGLU MLP block (the three matrices the page compresses, section "How
+ * to compress model weights effectively"; the block structure is not on the
+ * page): y = W_down (SiLU(W_gate x) * (W_up x)).  gate, up:
  * [ffn, d]; down: [d, ffn]; x: [batch, d]; y: [batch, d] (device BF16).
  * pipelines[3]: pipeline per matrix (gate, up, down), e.g. from uw_autotune.
  * The up GEMM applies SiLU(g)*u in its epilogue and writes h directly.
- * Workspace: uw_mlp_workspace_bytes. */
+ * Workspace: uw_mlp_workspace_bytes (0 for invalid arguments).  Errors:
+ * UW_ERR_INVALID_ARG (NULL pointers, or shapes that do not chain),
+ * UW_ERR_WORKSPACE_TOO_SMALL, and the errors of uw_gemm. */
 UW_API size_t uw_mlp_workspace_bytes(const uw_matrix* gate, const uw_matrix* up, const uw_matrix* down,
                               const int32_t* pipelines, int32_t batch);
 UW_API uw_status uw_mlp_block(const uw_matrix* gate, const uw_matrix* up, const uw_matrix* down,
@@ -380,7 +411,9 @@ UW_API uw_status uw_mlp_block(const uw_matrix* gate, const uw_matrix* up, const 
  * Autotuner (sections "Key Points" and "Why no single pipeline wins")
  * ------------------------------------------------------------------------- */
 
-/* Time every pipeline on this matrix at each batch and pick the fastest.
+/* Time every pipeline on this matrix at each batch and pick the fastest
+ * (sections "Key Points" and "Why no single pipeline wins": the best
+ * pipeline depends on the matrix shape and the batch).
  * For each batch b in batches[0..n_batches): warm up, then run reps timed
  * calls (CUDA events on `stream`, preprocessing included), and keep the
  * median.  out_us[i*4 + p] = median microseconds of pipeline p at batches[i]
@@ -391,7 +424,9 @@ UW_API uw_status uw_mlp_block(const uw_matrix* gate, const uw_matrix* up, const 
  * NULL/0): a device buffer larger than L2 that is overwritten before every
  * timed call so the weights are read from HBM as they are in a real decode
  * step.  Synchronizes `stream`.  Workspace: the maximum of
- * uw_workspace_bytes over the four pipelines and batches. */
+ * uw_workspace_bytes over the four pipelines and batches.  Errors:
+ * UW_ERR_INVALID_ARG (NULL outputs, n_batches or reps < 1), errors of the
+ * timed calls, UW_ERR_CUDA. */
 UW_API uw_status uw_autotune(const uw_matrix* m, const int32_t* batches, int32_t n_batches,
                       int32_t reps, const uint16_t* x, uint16_t* y, void* flush,
                       size_t flush_bytes, void* workspace, size_t workspace_bytes,
@@ -401,13 +436,15 @@ UW_API uw_status uw_autotune(const uw_matrix* m, const int32_t* batches, int32_t
  * Misc
  * ------------------------------------------------------------------------- */
 
+/* Human-readable name of a status code (library plumbing). */
 UW_API const char* uw_status_string(uw_status s);
 
-/* Library version: major*10000 + minor*100 + patch. */
+/* Library version: major*10000 + minor*100 + patch (library plumbing). */
 UW_API int32_t uw_version(void);
 
 /* Number of kernel launches the library has issued in this process (all
- * devices); used to count launches inside a timed region. */
+ * devices; library plumbing); used to count launches inside a timed
+ * region. */
 UW_API uint64_t uw_launch_count(void);
 
 #ifdef __cplusplus
