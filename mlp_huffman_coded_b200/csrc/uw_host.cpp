@@ -7,9 +7,12 @@
 // verbatim 64-element rows).  The storage layout is documented in uw.h.
 #include <algorithm>
 #include <array>
+#include <atomic>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <queue>
+#include <thread>
 #include <utility>
 #include <vector>
 
@@ -21,6 +24,35 @@ constexpr int kGroup = UW_GROUP;
 constexpr int kPal = UW_PALETTE;
 
 inline int popc32(uint32_t v) { return __builtin_popcount(v); }
+
+// Host threads for the encoder passes: every pass splits the 64-element
+// groups into contiguous ranges and combines per-thread results in a fixed
+// way, so the output is byte-identical for any thread count.  Small
+// matrices use one thread; UW_ENCODE_THREADS sets the count exactly.
+int encode_threads(int64_t n_groups) {
+  static const int env = [] {
+    const char* e = std::getenv("UW_ENCODE_THREADS");
+    return e ? std::atoi(e) : 0;
+  }();
+  if (env > 0) return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(env, n_groups)));
+  const int t = static_cast<int>(std::min(16u, std::max(1u, std::thread::hardware_concurrency())));
+  const int64_t by_size = n_groups / 16384 + 1;  // >= 1M elements per thread
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(t, by_size)));
+}
+
+// fn(thread, g_begin, g_end) over `nt` contiguous ranges of [0, n)
+template <class F>
+void for_ranges(int nt, int64_t n, F&& fn) {
+  if (nt <= 1) {
+    fn(0, int64_t(0), n);
+    return;
+  }
+  std::vector<std::thread> pool;
+  pool.reserve(nt);
+  for (int t = 0; t < nt; ++t)
+    pool.emplace_back([&, t] { fn(t, n * t / nt, n * (t + 1) / nt); });
+  for (auto& th : pool) th.join();
+}
 
 bool shape_ok(int64_t rows, int64_t cols) {
   return rows >= 1 && cols >= kGroup && cols % kGroup == 0 && rows <= (int64_t(1) << 40) / cols;
@@ -99,8 +131,17 @@ extern "C" uw_status uw_build_palette_codebook(const uint16_t* w, int64_t rows, 
   if (!w || !out) return UW_ERR_INVALID_ARG;
   if (!shape_ok(rows, cols)) return UW_ERR_UNSUPPORTED_SHAPE;
   const int64_t n = rows * cols;
+  const int64_t n_groups = n / kGroup;
+  const int nt = encode_threads(n_groups);
+  std::vector<std::array<uint64_t, 256>> part_hist(nt);
+  for_ranges(nt, n_groups, [&](int t, int64_t g0, int64_t g1) {
+    auto& h = part_hist[t];
+    h.fill(0);
+    for (int64_t i = g0 * kGroup; i < g1 * kGroup; ++i) ++h[(w[i] >> 7) & 0xFF];
+  });
   std::array<uint64_t, 256> hist{};
-  for (int64_t i = 0; i < n; ++i) ++hist[(w[i] >> 7) & 0xFF];
+  for (int t = 0; t < nt; ++t)
+    for (int e = 0; e < 256; ++e) hist[e] += part_hist[t][e];
   std::array<int, 256> order;
   for (int e = 0; e < 256; ++e) order[e] = e;
   std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
@@ -112,14 +153,20 @@ extern "C" uw_status uw_build_palette_codebook(const uint16_t* w, int64_t rows, 
   for (int i = 0; i < kPal; ++i) cb.palette[i] = static_cast<uint8_t>(order[i]);
   auto pm = palette_map(cb.palette);
   // frequencies over non-verbatim groups only
-  const int64_t n_groups = n / kGroup;
-  for (int64_t g = 0; g < n_groups; ++g) {
-    const uint16_t* p = w + g * kGroup;
-    bool verb = false;
-    for (int k = 0; k < kGroup; ++k) verb |= pm[(p[k] >> 7) & 0xFF] == 255;
-    if (verb) continue;
-    for (int k = 0; k < kGroup; ++k) ++cb.freq[pm[(p[k] >> 7) & 0xFF]];
-  }
+  std::vector<std::array<uint64_t, kPal>> part_freq(nt);
+  for_ranges(nt, n_groups, [&](int t, int64_t g0, int64_t g1) {
+    auto& f = part_freq[t];
+    f.fill(0);
+    for (int64_t g = g0; g < g1; ++g) {
+      const uint16_t* p = w + g * kGroup;
+      bool verb = false;
+      for (int k = 0; k < kGroup; ++k) verb |= pm[(p[k] >> 7) & 0xFF] == 255;
+      if (verb) continue;
+      for (int k = 0; k < kGroup; ++k) ++f[pm[(p[k] >> 7) & 0xFF]];
+    }
+  });
+  for (int t = 0; t < nt; ++t)
+    for (int i = 0; i < kPal; ++i) cb.freq[i] += part_freq[t][i];
   huffman_lengths(cb.freq, cb.code_len);
   canonical(cb.code_len, cb.code);
   int ns = 0, ml = 0;
@@ -147,27 +194,42 @@ extern "C" uw_status uw_encode(const uint16_t* w, int64_t rows, int64_t cols, co
   auto pm = palette_map(cb->palette);
 
   // pass 1: verbatim flags and coded bits per group
+  const int nt = encode_threads(n_groups);
   std::vector<uint8_t> verb(n_groups);
   std::vector<uint32_t> gbits(n_groups);
+  std::vector<uint64_t> part_bits(nt, 0);
+  std::vector<int64_t> part_verb(nt, 0);
+  std::atomic<bool> uncovered{false};
+  for_ranges(nt, n_groups, [&](int t, int64_t g0, int64_t g1) {
+    uint64_t bits = 0;
+    int64_t nv = 0;
+    for (int64_t g = g0; g < g1; ++g) {
+      const uint16_t* p = w + g * kGroup;
+      bool v = false;
+      for (int k = 0; k < kGroup; ++k) v |= pm[(p[k] >> 7) & 0xFF] == 255;
+      verb[g] = v;
+      uint32_t b = 0;
+      if (!v) {
+        for (int k = 0; k < kGroup; ++k) {
+          uint8_t len = cb->code_len[pm[(p[k] >> 7) & 0xFF]];
+          if (len == 0) uncovered = true;
+          b += len;
+        }
+      } else {
+        ++nv;
+      }
+      gbits[g] = b;
+      bits += b;
+    }
+    part_bits[t] = bits;
+    part_verb[t] = nv;
+  });
+  if (uncovered) return UW_ERR_CORRUPT;
   uint64_t total = 0;
   int64_t n_verb = 0;
-  for (int64_t g = 0; g < n_groups; ++g) {
-    const uint16_t* p = w + g * kGroup;
-    bool v = false;
-    for (int k = 0; k < kGroup; ++k) v |= pm[(p[k] >> 7) & 0xFF] == 255;
-    verb[g] = v;
-    uint32_t b = 0;
-    if (!v) {
-      for (int k = 0; k < kGroup; ++k) {
-        uint8_t len = cb->code_len[pm[(p[k] >> 7) & 0xFF]];
-        if (len == 0) return UW_ERR_CORRUPT;
-        b += len;
-      }
-    } else {
-      ++n_verb;
-    }
-    gbits[g] = b;
-    total += b;
+  for (int t = 0; t < nt; ++t) {
+    total += part_bits[t];
+    n_verb += part_verb[t];
   }
   if (total >= (uint64_t(1) << 32)) return UW_ERR_UNSUPPORTED_SHAPE;
 
@@ -188,12 +250,13 @@ extern "C" uw_status uw_encode(const uint16_t* w, int64_t rows, int64_t cols, co
     return UW_ERR_INVALID_ARG;
 
   // sign+mantissa bytes: own mantissa, pair partner's sign
-  const int64_t n = rows * cols;
-  for (int64_t i = 0; i < n; i += 2) {
-    uint16_t a = w[i], b = w[i + 1];
-    sm[i] = static_cast<uint8_t>(((a & 0x7F) << 1) | (b >> 15));
-    sm[i + 1] = static_cast<uint8_t>(((b & 0x7F) << 1) | (a >> 15));
-  }
+  for_ranges(nt, n_groups, [&](int, int64_t g0, int64_t g1) {
+    for (int64_t i = g0 * kGroup; i < g1 * kGroup; i += 2) {
+      uint16_t a = w[i], b = w[i + 1];
+      sm[i] = static_cast<uint8_t>(((a & 0x7F) << 1) | (b >> 15));
+      sm[i + 1] = static_cast<uint8_t>(((b & 0x7F) << 1) | (a >> 15));
+    }
+  });
 
   // chunk offsets
   uint64_t pos = 0;
@@ -203,26 +266,61 @@ extern "C" uw_status uw_encode(const uint16_t* w, int64_t rows, int64_t cols, co
   }
   chunk_bit_off[lay.n_chunks] = static_cast<uint32_t>(pos);
 
-  // bitstream, MSB first
+  // bitstream, MSB first.  Each thread packs a contiguous range of groups
+  // starting at its global bit offset (known from the group bit counts) into
+  // words aligned to the global word grid; it owns every word strictly
+  // inside its range, and the at most two words it shares with its
+  // neighbours are OR-ed in after all threads finish.
   std::memset(stream, 0, lay.stream_words * sizeof(uint32_t));
-  uint64_t acc = 0;  // pending bits, right aligned
-  int nacc = 0;
-  int64_t wi = 0;
-  for (int64_t g = 0; g < n_groups; ++g) {
-    if (verb[g]) continue;
-    const uint16_t* p = w + g * kGroup;
-    for (int k = 0; k < kGroup; ++k) {
-      int s = pm[(p[k] >> 7) & 0xFF];
-      acc = (acc << cb->code_len[s]) | cb->code[s];
-      nacc += cb->code_len[s];
-      if (nacc >= 32) {
-        stream[wi++] = static_cast<uint32_t>(acc >> (nacc - 32));
-        nacc -= 32;
-        acc &= (uint64_t(1) << nacc) - 1;
+  std::vector<uint64_t> start_bit(nt + 1, 0);
+  {
+    uint64_t b = 0;
+    for (int t = 0; t < nt; ++t) {
+      start_bit[t] = b;
+      b += part_bits[t];
+    }
+    start_bit[nt] = b;
+  }
+  struct Edge { int64_t word; uint32_t bits; };
+  std::vector<std::array<Edge, 2>> edges(nt, {Edge{-1, 0}, Edge{-1, 0}});
+  for_ranges(nt, n_groups, [&](int t, int64_t g0, int64_t g1) {
+    const uint64_t b0 = start_bit[t], b1 = start_bit[t + 1];
+    if (b1 == b0) return;
+    const int64_t first_word = static_cast<int64_t>(b0 / 32), last_word = static_cast<int64_t>((b1 - 1) / 32);
+    auto put = [&](int64_t wi, uint32_t v) {
+      // words this range shares with a neighbour go to the edge list
+      const bool shared_first = wi == first_word && (b0 % 32) != 0;
+      const bool shared_last = wi == last_word && (b1 % 32) != 0;
+      if (shared_first) {
+        edges[t][0] = Edge{wi, v};
+      } else if (shared_last) {
+        edges[t][1] = Edge{wi, v};
+      } else {
+        stream[wi] = v;
+      }
+    };
+    uint64_t acc = 0;  // pending bits, right aligned
+    int nacc = static_cast<int>(b0 % 32);  // leading zero bits: align to the word grid
+    int64_t wi = first_word;
+    for (int64_t g = g0; g < g1; ++g) {
+      if (verb[g]) continue;
+      const uint16_t* p = w + g * kGroup;
+      for (int k = 0; k < kGroup; ++k) {
+        int sym = pm[(p[k] >> 7) & 0xFF];
+        acc = (acc << cb->code_len[sym]) | cb->code[sym];
+        nacc += cb->code_len[sym];
+        if (nacc >= 32) {
+          put(wi++, static_cast<uint32_t>(acc >> (nacc - 32)));
+          nacc -= 32;
+          acc &= (uint64_t(1) << nacc) - 1;
+        }
       }
     }
-  }
-  if (nacc > 0) stream[wi++] = static_cast<uint32_t>(acc << (32 - nacc));
+    if (nacc > 0) put(wi++, static_cast<uint32_t>(acc << (32 - nacc)));
+  });
+  for (int t = 0; t < nt; ++t)
+    for (const Edge& e : edges[t])
+      if (e.word >= 0) stream[e.word] |= e.bits;
 
   // verbatim flags, per-word prefix counts, verbatim store
   std::memset(vflags, 0, sizeof(uint32_t) * rows * wpr);
