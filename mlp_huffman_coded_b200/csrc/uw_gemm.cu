@@ -22,11 +22,16 @@
 //    64 elements, i.e. exactly one 64-element group, so the verbatim check is
 //    one flag bit per row per k-block and never per element.
 //  * Persistent CTAs, one per SM, split the linearised (tile, k-block) space
-//    evenly (stream-K); a tile split across CTAs is reduced in CTA order by
-//    the last CTA to finish it, so the result does not depend on timing and
-//    is identical for every pipeline.
-//  * FP32 accumulators live in TMEM; the epilogue reads them with tcgen05.ld
-//    and rounds to nearest-even BF16 (optionally applying SiLU(g) * u).
+//    evenly (stream-K); a tile split across CTAs is finished by its first
+//    contributor, which adds the others' published partial sums to its own
+//    (still in TMEM) in CTA order, so the result does not depend on timing
+//    and is identical for every pipeline.
+//  * FP32 accumulators live in TMEM; the epilogue reads them with tcgen05.ld,
+//    rounds to nearest-even BF16 (optionally applying SiLU(g) * u) and writes
+//    16-row chunks through shared memory with TMA tensor stores.
+//  * Launches overlap the previous kernel on the stream (programmatic
+//    dependent launch): weights stream first; activations, outputs and the
+//    split-K counters wait for that kernel (griddepcontrol.wait).
 //  * Every barrier wait is bounded in time; a timeout records UW_ERR_TIMEOUT,
 //    drains in-flight copies and frees tensor memory before returning.
 #include <algorithm>
