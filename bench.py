@@ -37,8 +37,8 @@ HBM_FALLBACK_GBS = 6650.0
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch
 # of the direct-palette GEMM kernel (the 14336x4096 gate projection at batch 8,
-# ncu --set full; profiles/gemm_direct_palette_14336x4096_b8.md), valid only
-# for the kernel sources it was taken on: reported as null once they change.
+# from one ncu --set full capture), valid only for the kernel sources it was
+# taken on: reported as null once they change.
 NCU_TRAFFIC = {"bytes_per_launch": 93671936,
                "launch": "gate projection 14336x4096, batch 8",
                "sources_sha256": "682f3dec5e0ee4221e4987950b3c2ec2811d32554a1ddb771f7f3e7d7578910d"}
@@ -196,7 +196,8 @@ def oracle_prepare(batch: int, row_fraction: float):
 def oracle_block_sample(batch: int, row_fraction: float):
     """Oracle work for one step on a row sample of each matrix: rebuild W from
     the direct-palette form (sm + 4-bit indices + verbatim rows), float64
-    GEMM, SiLU(g) * u.  Returns the seconds scaled to the whole block."""
+    GEMM, SiLU(g) * u.  Returns (measured seconds, seconds scaled to the
+    whole block)."""
     from oracle import uw_oracle as O
     preps, xs = oracle_prepare(batch, row_fraction)
     t0 = time.perf_counter()
@@ -206,7 +207,7 @@ def oracle_block_sample(batch: int, row_fraction: float):
     _ = O.silu(outs[0]) * outs[1]
     dt = time.perf_counter() - t0
     frac = sum(f for _, _, f in preps) / 3
-    return dt / frac
+    return dt, dt / frac
 
 
 def run_reference(args, world, rank):
@@ -219,27 +220,34 @@ def run_reference(args, world, rank):
         for _ in range(args.warmup):
             oracle_block_sample(args.batch, frac)
         times = [oracle_block_sample(args.batch, frac) for _ in range(args.steps)]
-    step_s = sum(times) / len(times)   # full-block seconds per step
-    value = args.batch / step_s
+    sample_s = sum(t for t, _ in times) / len(times)     # measured seconds per (sample) step
+    full_s = sum(f for _, f in times) / len(times)       # the same scaled to the whole block
+    value = args.batch / full_s
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sample_s * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_dict(args),
+        "config": config_dict(args, world),
+        "ms_per_step_is": "measured time of one sample step (the rows below); value uses the full block",
+        "full_block_ms_per_step_extrapolated": full_s * 1e3,
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{frac:.4f} of the rows of gate, up and down per step, scaled to the full block"},
+                         "sample": f"each step: the first {frac:.4f} of the rows of gate, up and down "
+                                   f"(direct-palette rebuild + float64 GEMM + SiLU*up); tokens/s from its time "
+                                   f"scaled by the rows covered to the full block"},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
 
 
-def config_dict(args):
+def config_dict(args, world: int = 1):
+    """The workload, identical for the GPU arm and the oracle arm."""
     return {"workload": f"SwiGLU MLP block d={D_MODEL} ffn={FFN} (Llama-3.1-8B shapes), direct-palette "
                         f"reconstructive GEMM, batch {args.batch}",
             "batch": args.batch, "d_model": D_MODEL, "ffn": FFN, "pipeline": "direct palette (gate, up, down)",
             "weights": f"N(0,{SIGMA}) bf16, outliers {OUTLIER_RATE} x{OUTLIER_SCALE}, seed {SEED}",
-            "l2": "inputs larger than L2: 3 compressed matrices (~268 MB) streamed per step, L2 is 126 MB"}
+            "l2": "inputs larger than L2: 3 compressed matrices (~268 MB) streamed per step, L2 is 126 MB",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 
 # ---------------------------------------------------------------------------
@@ -346,10 +354,57 @@ def run_gpu(args, world, rank, local):
     # roofline of the dominant kernel (the reconstructive GEMM: every launch of
     # the step is one)
     peaks, src = measured_peaks()
-    per_step_bytes = sum(dm.direct_palette_bytes() for dm in dms) + 2 * B * (D_MODEL + FFN) * 2 + 2 * B * FFN * 2
+    peak = float(peaks["hbm_gbs"])
+    w_bytes = sum(dm.direct_palette_bytes() for dm in dms)
+
+    def step_bytes(b):
+        return w_bytes + 2 * b * (D_MODEL + FFN) * 2 + 2 * b * FFN * 2
+
+    per_step_bytes = step_bytes(B)
     t_step = ms / 1e3 / args.steps
     achieved = per_step_bytes / t_step / 1e9
-    peak = float(peaks["hbm_gbs"])
+
+    # the other batches the block is quoted at (1 and 32 next to the default
+    # 8): the same step, timed the same way, plus the BF16 comparator
+    other = {}
+    for b in [v for v in (1, 8, 32) if v != B]:
+        wsb = uw.Workspace(uw.mlp_workspace_bytes(*dms, pipes, b), device=dev)
+        xb_dev = torch.from_numpy(synth.activations(b, D_MODEL, 3).view(np.int16)).to(dev)
+        yb_dev = torch.empty(b, D_MODEL, dtype=torch.int16, device=dev)
+        for _ in range(args.warmup):
+            uw.mlp_block(*dms, pipes, xb_dev, yb_dev, wsb, stream)
+        torch.cuda.synchronize(dev)
+        n_b = max(3, args.steps)
+        h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h0.record(stream)
+        for _ in range(n_b):
+            uw.mlp_block(*dms, pipes, xb_dev, yb_dev, wsb, stream)
+        h1.record(stream)
+        h1.synchronize()
+        wsb.check(f"batch {b}")
+        ms_b = max_over_ranks(world, h0.elapsed_time(h1)) / n_b
+        wt_b = [torch.from_numpy(w.view(np.int16)).to(dev).view(torch.bfloat16) for w in mats]
+        xbb = xb_dev.view(torch.bfloat16)
+
+        def step_bf16_b():
+            g = xbb @ wt_b[0].T
+            u = xbb @ wt_b[1].T
+            return (torch.nn.functional.silu(g) * u) @ wt_b[2].T
+
+        for _ in range(3):
+            step_bf16_b()
+        torch.cuda.synchronize(dev)
+        h0.record(stream)
+        for _ in range(n_b):
+            step_bf16_b()
+        h1.record(stream)
+        h1.synchronize()
+        bf16_b = h0.elapsed_time(h1) / n_b
+        del wt_b
+        ach_b = step_bytes(b) / (ms_b / 1e3) / 1e9
+        other[str(b)] = {"ms_per_step": ms_b, "tokens_per_s": b * world / (ms_b / 1e3), "steps": n_b,
+                         "roofline_frac": ach_b / peak, "achieved_gbs": ach_b,
+                         "bf16_torch_matmul_ms_per_step": bf16_b, "speedup_vs_bf16_torch": bf16_b / ms_b}
     weight_gbs = sum(2 * e.rows * e.cols for e in encs) / t_step / 1e9
 
     if rank == 0:
@@ -366,7 +421,7 @@ def run_gpu(args, world, rank, local):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
-            "config": dict(config_dict(args), parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+            "config": config_dict(args, world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": ncu_traffic_per_launch(),
                          "traffic_launch": NCU_TRAFFIC["launch"],
@@ -374,6 +429,7 @@ def run_gpu(args, world, rank, local):
                                    "achieved = algorithmic bytes per step / step time)",
                          "algorithmic_bytes_per_step": per_step_bytes, "peak_source": f"{src} hbm_gbs"},
             "effective_weight_gbs": weight_gbs,
+            "other_batches": other,
             "bf16_torch_matmul_ms_per_step": bf16_ms,
             "speedup_vs_bf16_torch": bf16_ms / (ms / args.steps),
             "e2e": {"value": B * args.steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
@@ -385,7 +441,7 @@ def run_gpu(args, world, rank, local):
             from threadpoolctl import threadpool_limits
             with threadpool_limits(limits=1):
                 oracle_prepare(B, args.ref_fraction)
-                dt = min(oracle_block_sample(B, args.ref_fraction) for _ in range(3))
+                dt = min(oracle_block_sample(B, args.ref_fraction)[1] for _ in range(3))
             line["cpu_baseline"] = {
                 "value": B / dt, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                 "sample": f"best of 3 steps on {args.ref_fraction:.4f} of the rows of gate, up and down "

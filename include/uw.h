@@ -49,25 +49,27 @@
  *               byte j of the row, 2j+1 in the high nibble; 0 in verbatim
  *               groups.
  *   pack        (optional, the direct-palette form built at load time by
- *               uw_pack_direct_palette) one contiguous record per tile of
- *               128 rows x 64 columns, tiles in (row block, column block)
- *               order, record t starting at byte 16*pack_off[t]:
+ *               uw_pack_direct_palette) for the n_tiles = ceil(rows/128) *
+ *               cols/64 tiles of 128 rows x 64 columns, in (row block,
+ *               column block) order: first one fixed-size 12304-byte body
+ *               per tile, body t at byte 12304*t:
  *                 [0, 8192)      sm bytes of the tile: row r, 16-byte chunk
  *                                j at r*64 + 16*(j ^ ((r>>1)&3))
  *                 [8192, 12288)  idx4 bytes of the tile: row r, chunk j at
  *                                8192 + r*32 + 16*(j ^ ((r>>2)&1))
  *                 [12288, 12304) 128-bit verbatim mask, bit r = row r's
  *                                64-element group is verbatim
- *                 [12304, 12416) zero (keeps every record 128-byte aligned)
- *                 [12416, ...)   the first min(n, 32) verbatim rows of the
- *                                tile (64 BF16 words each), in row order
- *               Rows past `rows` are zero.  A tile with more than 32 verbatim
- *               rows keeps the rest in the verbatim store only.  The chunk
+ *               then, from byte 12304*n_tiles, the verbatim rows of every
+ *               tile (64 BF16 words = 128 bytes each) in tile order and, in a
+ *               tile, in row order.  Rows past `rows` are zero.  The chunk
  *               order inside each 64-/32-byte row is the one that makes the
  *               GEMM's row-per-thread 16-byte shared-memory reads free of
- *               bank conflicts.
- *   pack_off    uint32[n_tiles+1]: record offsets in 16-byte units
- *               (uw_direct_pack_offsets), n_tiles = ceil(rows/128)*cols/64.
+ *               bank conflicts; fixed-size bodies let the GEMM fetch several
+ *               consecutive tiles with one copy whose address it computes.
+ *   pack_off    uint32[n_tiles+1]: pack_off[t] = verbatim rows of all tiles
+ *               before t, so tile t's verbatim rows start at byte
+ *               12304*n_tiles + 128*pack_off[t]; the last entry is n_verbatim
+ *               (uw_direct_pack_offsets).
  *
  * Conventions for every call:
  *   - Every call returns a uw_status; nothing throws across the ABI.
@@ -210,13 +212,14 @@ UW_API uw_status uw_encode(const uint16_t* w_host, int64_t rows, int64_t cols, c
                     uint32_t* chunk_bit_off, uint32_t* vflags, uint32_t* vprefix,
                     uint16_t* verbatim);
 
-/* Record offsets (16-byte units) of the direct-palette pack of a matrix
- * (section "How the reconstructive matmul works": what the producer stages
- * per tile -- sign+mantissa bytes, palette indices, verbatim rows; the byte
- * layout is this library's), computed from its HOST vflags: pack_off[t+1] - pack_off[t] =
- * (12416 + 128*min(verbatim rows of tile t, 32)) / 16.  pack_off_host holds
- * n_tiles+1 entries; *pack_bytes (may be NULL) receives the total size.
- * Errors: UW_ERR_INVALID_ARG, UW_ERR_UNSUPPORTED_SHAPE (pack above 64 GiB). */
+/* Verbatim-row offsets of the direct-palette pack of a matrix (section "How
+ * the reconstructive matmul works": what the producer stages per tile --
+ * sign+mantissa bytes, palette indices, verbatim rows; the byte layout is
+ * this library's), computed from its HOST vflags: pack_off[t] = verbatim
+ * groups of all tiles before t.  pack_off_host holds n_tiles+1 entries;
+ * *pack_bytes (may be NULL) receives the pack's size, 12304*n_tiles +
+ * 128*n_verbatim.  Errors: UW_ERR_INVALID_ARG, UW_ERR_CORRUPT
+ * (words_per_row), UW_ERR_UNSUPPORTED_SHAPE (pack above 64 GiB). */
 UW_API uw_status uw_direct_pack_offsets(const uw_layout* L, const uint32_t* vflags_host,
                                         uint32_t* pack_off_host, uint64_t* pack_bytes);
 
@@ -240,17 +243,22 @@ UW_API uw_status uw_validate(const uw_matrix* host_mirror);
  * for invalid arguments. */
 UW_API size_t uw_workspace_bytes(const uw_layout* L, int32_t pipeline, int32_t batch);
 
-/* Zero a workspace (stream-ordered; library plumbing).  A workspace must be
- * zeroed once before its first use; afterwards every call leaves its
- * counters at zero again.  Calls that share one workspace must be ordered on
- * one stream.  Errors: UW_ERR_INVALID_ARG (NULL, misaligned, < 256 bytes),
- * UW_ERR_CUDA. */
+/* Zero a workspace and record its size in its header (library plumbing;
+ * synchronizes `stream`).  A workspace must be set up once before its first
+ * use; afterwards every call that succeeds leaves its counters at zero
+ * again, and a call that fails is cleaned up by uw_workspace_status.  Calls
+ * that share one workspace must be ordered on one stream.  Errors:
+ * UW_ERR_INVALID_ARG (NULL, misaligned, < 256 bytes), UW_ERR_CUDA. */
 UW_API uw_status uw_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronize the stream, read the workspace's sticky status word (the
  * first problem any kernel recorded since the last read) and clear it
- * (library plumbing).  Returns that status (UW_OK when none), or
- * UW_ERR_INVALID_ARG / UW_ERR_CUDA for the read itself. */
+ * (library plumbing).  When it is not UW_OK, a kernel gave up part way and
+ * may have left split-K tile counters raised, so the whole workspace is
+ * zeroed again (the size recorded by uw_workspace_init; a workspace zeroed
+ * some other way must be zeroed again by the caller before its next use).
+ * Returns that status (UW_OK when none), or UW_ERR_INVALID_ARG / UW_ERR_CUDA
+ * for the read itself. */
 UW_API uw_status uw_workspace_status(void* workspace, void* stream);
 
 /* Self-test of the bounded waits (no counterpart on the page: a robustness
@@ -359,8 +367,9 @@ UW_API uw_status uw_gemm_direct_palette_general_lookup(const uw_matrix* m, const
  *   - Every GPU that loads the library holds that 16 MiB until exit.
  *   - Limit: header + tile counters + split-K partials must fit in it, i.e.
  *     (ceil(rows/128)*ceil(batch/256) + SMs) * batch_tile * 512 bytes plus a
- *     few KB; a 14336 x 4096 matrix fits up to batch 64.  Larger sizes return
- *     UW_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *     few KB, batch_tile = batch rounded up to a multiple of 16 (per 256);
+ *     on a 148-SM B200 a 14336 x 4096 matrix fits up to batch 112.  Larger
+ *     sizes return UW_ERR_WORKSPACE_TOO_SMALL before anything is launched.
  *   - The first call on a device looks the array's device address up
  *     (cudaGetSymbolAddress); make that first call before any stream
  *     capture.

@@ -44,6 +44,7 @@ struct DecodeParams {
   void* out;
   uint32_t* status;
   int64_t n_groups;
+  int64_t n_verbatim;
   int64_t n_chunks;
   int64_t stream_words;
   int32_t chunk_groups;
@@ -171,17 +172,25 @@ __global__ void __launch_bounds__(kDecodeThreads, 7) decode_kernel(const DecodeP
       const int64_t e0 = g * 64;
       if (flags & bit) {
         // verbatim group: raw words from the store, no stream bits
-        const int64_t slot = __ldg(p.vprefix + fw) + __popc(flags & (bit - 1));
+        int64_t slot = __ldg(p.vprefix + fw) + __popc(flags & (bit - 1));
+        if (slot >= p.n_verbatim) {
+          // corrupt flags or prefixes: report, and read nothing outside the
+          // store (slot 0 stands in; a store-less matrix writes zeros)
+          record_status(p.status, UW_ERR_CORRUPT);
+          slot = 0;
+        }
+        const bool have = p.n_verbatim > 0;
+        const uint4 zero = make_uint4(0, 0, 0, 0);
         const uint4* src = reinterpret_cast<const uint4*>(p.verbatim + slot * 64);
         if (MODE == kFull) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + e0);
 #pragma unroll
-          for (int k = 0; k < 8; ++k) dst[k] = __ldg(src + k);
+          for (int k = 0; k < 8; ++k) dst[k] = have ? __ldg(src + k) : zero;
         } else if (MODE == kExp8) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + e0);
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint4 a = __ldg(src + 2 * k), b = __ldg(src + 2 * k + 1);
+            const uint4 a = have ? __ldg(src + 2 * k) : zero, b = have ? __ldg(src + 2 * k + 1) : zero;
             // exponent = bits 7..14 of each 16-bit word: take the byte that
             // straddles them after a 7-bit right shift of each word pair
             const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
@@ -290,6 +299,7 @@ uw_status launch_decode(const uw_matrix* m, int mode, void* out, uint32_t* statu
   p.out = out;
   p.status = status;
   p.n_groups = m->L.n_groups;
+  p.n_verbatim = m->L.n_verbatim;
   p.n_chunks = m->L.n_chunks;
   p.stream_words = m->L.stream_words;
   p.chunk_groups = m->L.chunk_groups;

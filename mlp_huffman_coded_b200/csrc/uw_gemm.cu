@@ -16,16 +16,22 @@
 //    N = 16 MMA.
 //  * Rebuilt BF16 goes from registers into tensor memory (tcgen05.st) and the
 //    MMA reads A from TMEM; shared memory only carries the compressed tiles
-//    and the activation tile.  This keeps shared-memory traffic near 2.3
-//    bytes per weight instead of ~7 with an SMEM round trip.
+//    and the activation tile.
 //  * One rebuild thread owns one weight row (= one TMEM lane) per k-block of
 //    64 elements, i.e. exactly one 64-element group, so the verbatim check is
 //    one flag bit per row per k-block and never per element.
+//  * A pipeline stage carries `ks` consecutive k-blocks of one row tile: one
+//    bulk copy brings all their direct-palette records (fixed-size bodies, so
+//    their address needs no lookup) and one 3-D TMA load their activation
+//    tiles, so the per-stage costs of the producer and the MMA issuer (copy
+//    issue, barrier waits, tcgen05.commit) are paid once per `ks` k-blocks.
+//    The producer is one thread running a short loop; the weight copies of
+//    the first stages leave before any table is read.
 //  * Persistent CTAs, one per SM, split the linearised (tile, k-block) space
 //    evenly (stream-K); a tile split across CTAs is finished by its first
 //    contributor, which adds the others' published partial sums to its own
 //    (still in TMEM) in CTA order, so the result does not depend on timing
-//    and is identical for every pipeline.
+//    and is identical for every pipeline and stage size.
 //  * FP32 accumulators live in TMEM; the epilogue reads them with tcgen05.ld,
 //    rounds to nearest-even BF16 (optionally applying SiLU(g) * u) and writes
 //    16-row chunks through shared memory with TMA tensor stores.
@@ -47,16 +53,17 @@ namespace uw {
 namespace {
 
 // Warp roles: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), then
-// `groups` rebuild warpgroups of 4 warps (group g rebuilds the stages of
-// units i with i % groups == g, so several stages are rebuilt at once), then
-// 4 epilogue warps.
+// `groups` rebuild warpgroups of 4 warps (group g rebuilds stages i with
+// i % groups == g, so several stages are rebuilt at once), then 4 epilogue
+// warps.
 constexpr int kMaxGroups = 2;
 constexpr int kMaxThreads = 32 * (6 + 4 * kMaxGroups);
 constexpr int kWarpProducer = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWarpRebuild0 = 2;
-constexpr int kVCap = 16;         // verbatim rows staged on chip per tile
+constexpr int kVCap = 16;  // run-time transcode: verbatim rows staged per k-block
 constexpr int kMaxStages = 16;
+constexpr int kMaxKS = 4;  // k-blocks per stage
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;  // accumulators first; rebuilt A tiles after them
 constexpr size_t kSmemLimit = 227 * 1024;
@@ -65,28 +72,31 @@ constexpr size_t kSmemFloor = 120 * 1024;  // keeps one CTA (and one TMEM owner)
 // Tile loaders: BF16 tiles (full-decode pipeline and the uncompressed
 // comparator), sm + exponent bytes (exponent-only pipeline), row-major sm +
 // 4-bit indices + verbatim store (run-time transcode pipeline) and the
-// direct-palette pack records; U/M = palette lookup for a uniform / mixed
-// top exponent bit.
+// direct-palette pack; U/M = palette lookup for a uniform / mixed top
+// exponent bit.
 enum KernelLoader { kBF16 = 0, kEXP8 = 1, kIDX4U = 2, kIDX4M = 3, kPACKU = 4, kPACKM = 5 };
 __host__ __device__ constexpr bool loader_pack(int L) { return L == kPACKU || L == kPACKM; }
+__host__ __device__ constexpr bool loader_idx4(int L) { return L == kIDX4U || L == kIDX4M; }
 __host__ __device__ constexpr bool loader_uniform(int L) { return L == kIDX4U || L == kPACKU; }
-constexpr uint32_t kRecIdx = 8192, kRecMask = 12288, kRecVerb = 12416, kRecVCap = 32;
-constexpr uint32_t kRecMax = kRecVerb + kRecVCap * 128;
-constexpr uint32_t kPackMinVCap = 4;  // verbatim rows staged on chip per tile, at least
+// direct-palette pack body of one 128 x 64 tile (layout in uw.h)
+constexpr uint32_t kBody = 12304, kBodyIdx = 8192, kBodyMask = 12288;
+constexpr uint32_t kPackMinTail = 4;  // verbatim rows staged on chip per stage, at least
 
 struct KParams {
   int N, K, B, KB, n_ntiles, ntile;
   long long units;
   int grid;
   int stages;
+  int ks;  // k-blocks per stage
   uint32_t stage_bytes, off_x, off_wa, off_wb, off_verb, off_hdr;
-  uint32_t x_bytes, wa_bytes, wb_bytes;
-  uint32_t meta_off, meta_slot_words;  // per slot: flags then prefixes
+  uint32_t x_kb_bytes;  // activation tile of one k-block: ntile rows x 128 bytes
+  uint32_t meta_off, meta_slot_words;  // run-time transcode: per slot flags then prefixes
   uint32_t bar_off;
   int wpr;
   const uint32_t* vflags;
   const uint32_t* vprefix;
   const uint16_t* verbatim;
+  long long n_verbatim;
   uint16_t* y;
   const uint16_t* gate;
   float* partials;
@@ -95,16 +105,17 @@ struct KParams {
   PaletteTables pal;
   uint32_t idesc;
   int groups;  // rebuild warpgroups
-  int vcap;    // verbatim rows staged on chip per tile
+  int vcap;    // verbatim rows staged on chip: per stage (pack) / per k-block (transcode)
   int n_acc;   // accumulator buffers in TMEM (2 alternate segments when they fit)
-  const uint8_t* pack;
-  const uint32_t* pack_off;
-  uint32_t off_rec;   // pack record inside a stage
-  uint32_t soff_off;  // shared-memory copy of this CTA's record offsets
+  const uint8_t* pack;       // pack bodies
+  const uint8_t* tails;      // pack verbatim rows, tile order
+  const uint32_t* pack_off;  // per tile: verbatim rows of all earlier tiles
+  uint32_t soff_off;  // shared-memory copy of this CTA's pack_off entries
   int n_soff;         // its capacity in words
-  uint32_t a_col0;    // first TMEM column of the rebuilt A tiles (32 per stage)
+  uint32_t a_col0;    // first TMEM column of the rebuilt A tiles (32 per k-block)
   uint32_t epi_off;   // epilogue staging: 2 output chunks (+ 2 gate chunks)
   int tma_out;        // outputs leave through TMA tensor stores (else per element)
+  int x3d;            // a stage's activation tiles arrive in one 3-D TMA load
 };
 
 struct Bars {
@@ -126,6 +137,41 @@ __device__ __forceinline__ int64_t unit_begin(int64_t c, const KParams& p) {
 // CTA whose unit range holds unit u
 __device__ __forceinline__ int64_t unit_owner(int64_t u, const KParams& p) {
   return ((u + 1) * p.grid - 1) / p.units;
+}
+
+// Walks a CTA's stages in order: a stage is up to `ks` consecutive k-blocks
+// of one (row tile, batch tile); it never crosses a tile or the CTA's range.
+// Every role walks the same sequence; advancing costs no division.
+struct StageWalk {
+  int64_t u;  // first unit of the stage
+  int kb;     // its k-block
+  int mt, nt;
+  int n;  // k-blocks in the stage
+};
+__device__ __forceinline__ void walk_fix_n(StageWalk& w, int64_t u1, const KParams& p) {
+  const int64_t left = u1 - w.u;
+  const int lim = p.KB - w.kb < p.ks ? p.KB - w.kb : p.ks;
+  w.n = left < lim ? static_cast<int>(left) : lim;
+}
+__device__ __forceinline__ void walk_init(StageWalk& w, int64_t u0, int64_t u1, const KParams& p) {
+  const int64_t t = u0 / p.KB;
+  w.u = u0;
+  w.kb = static_cast<int>(u0 - t * p.KB);
+  w.mt = static_cast<int>(t / p.n_ntiles);
+  w.nt = static_cast<int>(t - static_cast<int64_t>(w.mt) * p.n_ntiles);
+  walk_fix_n(w, u1, p);
+}
+__device__ __forceinline__ void walk_next(StageWalk& w, int64_t u1, const KParams& p) {
+  w.u += w.n;
+  w.kb += w.n;
+  if (w.kb == p.KB) {
+    w.kb = 0;
+    if (++w.nt == p.n_ntiles) {
+      w.nt = 0;
+      ++w.mt;
+    }
+  }
+  walk_fix_n(w, u1, p);
 }
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* b, uint32_t* status) {
@@ -158,68 +204,96 @@ __device__ __forceinline__ void store_out(const KParams& p, int b, int64_t n, fl
   reinterpret_cast<__nv_bfloat16*>(p.y)[i] = val;
 }
 
+// Word q (0..3) of a 128-bit row mask, and the rows set in the words below it.
+__device__ __forceinline__ uint32_t mask_word(const uint4& m, int q) {
+  return q == 0 ? m.x : (q == 1 ? m.y : (q == 2 ? m.z : m.w));
+}
+__device__ __forceinline__ int mask_below(const uint4& m, int q) {
+  return (q > 0 ? __popc(m.x) : 0) + (q > 1 ? __popc(m.y) : 0) + (q > 2 ? __popc(m.z) : 0);
+}
+
 // ----------------------------- tile rebuild ---------------------------------
 // Each rebuild thread owns one row r of the 128-row tile and produces the 64
-// BF16 values of the current k-block as 32 packed words (element 2i in the
-// low half of word i), ready for tcgen05.st.  Tile rows come from TMA with a
-// swizzle that keeps these row-per-thread 16-byte reads bank-conflict free.
+// BF16 values of k-block j of the current stage as 32 packed words (element
+// 2i in the low half of word i), ready for tcgen05.st.  Tile rows arrive with
+// a swizzle that keeps these row-per-thread 16-byte reads bank-conflict free.
+
+__device__ __forceinline__ void rebuild_idx_row(const PaletteTables& pal, bool uniform, const uint8_t* ts,
+                                                const uint8_t* ti, int r, uint32_t (&o)[32]) {
+  uint32_t iw[8];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const uint4 v = lds128(ti + r * 32 + ((j ^ ((r >> 2) & 1)) << 4));
+    iw[4 * j] = v.x;
+    iw[4 * j + 1] = v.y;
+    iw[4 * j + 2] = v.z;
+    iw[4 * j + 3] = v.w;
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint4 s = lds128(ts + r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
+    const uint32_t sw[4] = {s.x, s.y, s.z, s.w};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t nib = iw[2 * j + h];  // 8 indices: elements 16j + 8h .. +7
+      uint32_t e0, e1;
+      if (uniform) {
+        e0 = lookup4_uniform(pal, nib);
+        e1 = lookup4_uniform(pal, nib >> 16);
+      } else {
+        e0 = lookup4_mixed(pal, nib);
+        e1 = lookup4_mixed(pal, nib >> 16);
+      }
+      rebuild4(sw[2 * h], e0, o[8 * j + 4 * h + 0], o[8 * j + 4 * h + 1]);
+      rebuild4(sw[2 * h + 1], e1, o[8 * j + 4 * h + 2], o[8 * j + 4 * h + 3]);
+    }
+  }
+}
 
 template <int L>
-__device__ __forceinline__ void rebuild_row(const uint8_t* stage, const KParams& p, int r, uint32_t (&o)[32]) {
+__device__ __forceinline__ void rebuild_row(const uint8_t* stage, const KParams& p, int r, int j,
+                                            uint32_t (&o)[32]) {
   if constexpr (L == kBF16) {
-    const uint8_t* t = stage + p.off_wa;  // rows of 128 B, 128-byte swizzle
+    const uint8_t* t = stage + p.off_wa + j * 16384;  // rows of 128 B, 128-byte swizzle
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint4 v = lds128(t + r * 128 + ((j ^ (r & 7)) << 4));
-      o[4 * j] = v.x;
-      o[4 * j + 1] = v.y;
-      o[4 * j + 2] = v.z;
-      o[4 * j + 3] = v.w;
+    for (int c = 0; c < 8; ++c) {
+      const uint4 v = lds128(t + r * 128 + ((c ^ (r & 7)) << 4));
+      o[4 * c] = v.x;
+      o[4 * c + 1] = v.y;
+      o[4 * c + 2] = v.z;
+      o[4 * c + 3] = v.w;
     }
   } else if constexpr (L == kEXP8) {
-    const uint8_t* ts = stage + p.off_wa;  // sm rows of 64 B, 64-byte swizzle
-    const uint8_t* te = stage + p.off_wb;  // exponent rows of 64 B, 64-byte swizzle
+    const uint8_t* ts = stage + p.off_wa + j * 8192;  // sm rows of 64 B, 64-byte swizzle
+    const uint8_t* te = stage + p.off_wb + j * 8192;  // exponent rows of 64 B, 64-byte swizzle
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = (j ^ ((r >> 1) & 3)) << 4;
-      const uint4 s = lds128(ts + r * 64 + c);
-      const uint4 e = lds128(te + r * 64 + c);
-      rebuild4(s.x, e.x, o[8 * j + 0], o[8 * j + 1]);
-      rebuild4(s.y, e.y, o[8 * j + 2], o[8 * j + 3]);
-      rebuild4(s.z, e.z, o[8 * j + 4], o[8 * j + 5]);
-      rebuild4(s.w, e.w, o[8 * j + 6], o[8 * j + 7]);
+    for (int c = 0; c < 4; ++c) {
+      const int off = (c ^ ((r >> 1) & 3)) << 4;
+      const uint4 s = lds128(ts + r * 64 + off);
+      const uint4 e = lds128(te + r * 64 + off);
+      rebuild4(s.x, e.x, o[8 * c + 0], o[8 * c + 1]);
+      rebuild4(s.y, e.y, o[8 * c + 2], o[8 * c + 3]);
+      rebuild4(s.z, e.z, o[8 * c + 4], o[8 * c + 5]);
+      rebuild4(s.w, e.w, o[8 * c + 6], o[8 * c + 7]);
     }
+  } else if constexpr (loader_pack(L)) {
+    const uint8_t* body = stage + p.off_wa + j * kBody;
+    rebuild_idx_row(p.pal, loader_uniform(L), body, body + kBodyIdx, r, o);
   } else {
-    const uint8_t* ts = stage + p.off_wa;  // sm rows of 64 B, 64-byte swizzle
-    const uint8_t* ti = stage + p.off_wb;  // index rows of 32 B, 32-byte swizzle
-    uint32_t iw[8];
+    // run-time transcode: sm rows of 64 B (64-byte swizzle), index rows of
+    // 32 B (32-byte swizzle)
+    rebuild_idx_row(p.pal, loader_uniform(L), stage + p.off_wa + j * 8192, stage + p.off_wb + j * 4096, r, o);
+  }
+}
+
+__device__ __forceinline__ void copy_row(const uint4* src, uint32_t (&o)[32]) {
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const uint4 v = lds128(ti + r * 32 + ((j ^ ((r >> 2) & 1)) << 4));
-      iw[4 * j] = v.x;
-      iw[4 * j + 1] = v.y;
-      iw[4 * j + 2] = v.z;
-      iw[4 * j + 3] = v.w;
-    }
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint4 s = lds128(ts + r * 64 + ((j ^ ((r >> 1) & 3)) << 4));
-      const uint32_t sw[4] = {s.x, s.y, s.z, s.w};
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t nib = iw[2 * j + h];  // 8 indices: elements 16j + 8h .. +7
-        uint32_t e0, e1;
-        if constexpr (loader_uniform(L)) {
-          e0 = lookup4_uniform(p.pal, nib);
-          e1 = lookup4_uniform(p.pal, nib >> 16);
-        } else {
-          e0 = lookup4_mixed(p.pal, nib);
-          e1 = lookup4_mixed(p.pal, nib >> 16);
-        }
-        rebuild4(sw[2 * h], e0, o[8 * j + 4 * h + 0], o[8 * j + 4 * h + 1]);
-        rebuild4(sw[2 * h + 1], e1, o[8 * j + 4 * h + 2], o[8 * j + 4 * h + 3]);
-      }
-    }
+  for (int c = 0; c < 8; ++c) {
+    const uint4 v = src[c];
+    o[4 * c] = v.x;
+    o[4 * c + 1] = v.y;
+    o[4 * c + 2] = v.z;
+    o[4 * c + 3] = v.w;
   }
 }
 
@@ -229,7 +303,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_wa,
                 const __grid_constant__ CUtensorMap tm_wb, const __grid_constant__ CUtensorMap tm_y,
                 const __grid_constant__ CUtensorMap tm_g, const KParams p) {
-  constexpr bool kIdx4 = (L == kIDX4U || L == kIDX4M);  // row-major indices + verbatim store
+  constexpr bool kIdx4 = loader_idx4(L);  // row-major indices + verbatim store
   constexpr bool kPack = loader_pack(L);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -244,62 +318,112 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 
   const int mt_first = static_cast<int>((u0 / p.KB) / p.n_ntiles);
   const int mt_last = static_cast<int>(((u1 - 1) / p.KB) / p.n_ntiles);
-  // pack records: this CTA's record offsets, loaded first of all (by the
-  // producer warp, while the MMA warp sets up barriers and tensor memory) --
-  // the first weight copy waits for them
   uint32_t* soff = reinterpret_cast<uint32_t*>(smem + p.soff_off);
   const int64_t pt_min = static_cast<int64_t>(mt_first) * p.KB;
-  if (kPack && warp == kWarpProducer) {
-    const int64_t n_tiles_total = static_cast<int64_t>((p.N + 127) / 128) * p.KB;
-    const int64_t want = static_cast<int64_t>(mt_last - mt_first + 1) * p.KB + 1;
-    const int64_t cnt = want < p.n_soff ? want : p.n_soff;
-    // all loads of a 256-word chunk are in flight before the first store:
-    // one memory round trip per chunk instead of one per word and lane
-    for (int64_t w0 = 0; w0 < cnt; w0 += 256) {
-      uint32_t v[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int64_t w = w0 + j * 32 + lane;
-        v[j] = (w < cnt && pt_min + w <= n_tiles_total) ? __ldg(p.pack_off + pt_min + w) : 0u;
+
+  // Weight bytes of a stage, and their copies (every loader but the run-time
+  // transcode, whose verbatim rows need the flag tables first).
+  auto weight_bytes = [&](const StageWalk& w) -> uint32_t {
+    if constexpr (kPack) return static_cast<uint32_t>(w.n) * kBody;
+    else if constexpr (L == kBF16) return static_cast<uint32_t>(w.n) * 16384u;
+    else return static_cast<uint32_t>(w.n) * (kIdx4 ? 12288u : 16384u);
+  };
+  const uint64_t stream_policy = l2_evict_first();
+  auto issue_weights = [&](int s, const StageWalk& w) {
+    uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
+    if constexpr (kPack) {
+      const int64_t tile = static_cast<int64_t>(w.mt) * p.KB + w.kb;
+      bulk_load_hint(stage + p.off_wa, p.pack + static_cast<uint64_t>(tile) * kBody, static_cast<uint32_t>(w.n) * kBody,
+                     &bars->full[s], stream_policy);
+    } else {
+      for (int j = 0; j < w.n; ++j) {
+        const int c = (w.kb + j) * 64;
+        if constexpr (L == kBF16) {
+          tma_load_2d(stage + p.off_wa + j * 16384, &tm_wa, c, w.mt * 128, &bars->full[s]);
+        } else if constexpr (L == kEXP8) {
+          tma_load_2d(stage + p.off_wa + j * 8192, &tm_wa, c, w.mt * 128, &bars->full[s]);
+          tma_load_2d(stage + p.off_wb + j * 8192, &tm_wb, c, w.mt * 128, &bars->full[s]);
+        } else {
+          tma_load_2d(stage + p.off_wa + j * 8192, &tm_wa, c, w.mt * 128, &bars->full[s]);
+          tma_load_2d(stage + p.off_wb + j * 4096, &tm_wb, c / 2, w.mt * 128, &bars->full[s]);
+        }
       }
+    }
+  };
+  auto issue_x = [&](int s, const StageWalk& w) {
+    uint8_t* dst = smem + static_cast<size_t>(s) * p.stage_bytes + p.off_x;
+    if (p.x3d) {
+      tma_load_3d(dst, &tm_x, 0, w.nt * p.ntile, w.kb, &bars->full[s]);
+    } else {
+      for (int j = 0; j < p.ks; ++j)
+        tma_load_2d(dst + j * p.x_kb_bytes, &tm_x, (w.kb + j) * 64, w.nt * p.ntile, &bars->full[s]);
+    }
+  };
+
+  // ---- set-up.  The producer thread initialises the barriers and at once
+  // issues the weight copies of the first stages (their phases cannot
+  // complete before its own arrive, which follows once the tables are in);
+  // the MMA warp allocates tensor memory meanwhile.
+  int early = 0;  // stages whose weights are already in flight
+  if (warp == kWarpProducer) {
+    if (lane == 0) {
+      for (int s = 0; s < S; ++s) {
+        mbar_init(&bars->full[s], 1);
+        mbar_init(&bars->rebuilt[s], 4);
+        mbar_init(&bars->empty[s], 1);
+      }
+      mbar_init(&bars->acc_full[0], 1);
+      mbar_init(&bars->acc_full[1], 1);
+      mbar_init(&bars->acc_empty[0], 4);
+      mbar_init(&bars->acc_empty[1], 4);
+      mbar_init(&bars->drain, 1);
+      mbar_init(&bars->meta_full[0], 1);
+      mbar_init(&bars->meta_full[1], 1);
+      mbar_init(&bars->gate_full[0], 1);
+      mbar_init(&bars->gate_full[1], 1);
+      bars->abort = 0;
+      bars->is_last = 0;
+      bars->dep_ready = 0;
+      mbar_fence_init();
+      if constexpr (!kIdx4) {
+        StageWalk w;
+        walk_init(w, u0, u1, p);
+        for (; early < S && w.u < u1; ++early, walk_next(w, u1, p)) {
+          mbar_expect_tx(&bars->full[early], weight_bytes(w));
+          issue_weights(early, w);
+        }
+      }
+      prefetch_tensormap(&tm_x);
+      if (p.tma_out) prefetch_tensormap(&tm_y);
+      if (p.tma_out && p.gate) prefetch_tensormap(&tm_g);
+      if (!kPack) prefetch_tensormap(&tm_wa);
+      if (L != kBF16 && !kPack) prefetch_tensormap(&tm_wb);
+    }
+    early = __shfl_sync(0xFFFFFFFFu, early, 0);
+    // pack: this CTA's pack_off entries (verbatim-row offsets of its tiles)
+    if (kPack) {
+      const int64_t n_tiles_total = static_cast<int64_t>((p.N + 127) / 128) * p.KB;
+      const int64_t want = static_cast<int64_t>(mt_last - mt_first + 1) * p.KB + 1;
+      const int64_t cnt = want < p.n_soff ? want : p.n_soff;
+      for (int64_t w0 = 0; w0 < cnt; w0 += 256) {
+        uint32_t v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int64_t w = w0 + j * 32 + lane;
-        if (w < cnt) soff[w] = v[j];
+        for (int j = 0; j < 8; ++j) {
+          const int64_t w = w0 + j * 32 + lane;
+          v[j] = (w < cnt && pt_min + w <= n_tiles_total) ? __ldg(p.pack_off + pt_min + w) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int64_t w = w0 + j * 32 + lane;
+          if (w < cnt) soff[w] = v[j];
+        }
       }
     }
     __syncwarp();
   }
-  if (threadIdx.x == 32 * kWarpMma) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(&bars->full[s], 1);
-      mbar_init(&bars->rebuilt[s], 4);
-      mbar_init(&bars->empty[s], 1);
-    }
-    mbar_init(&bars->acc_full[0], 1);
-    mbar_init(&bars->acc_full[1], 1);
-    mbar_init(&bars->acc_empty[0], 4);
-    mbar_init(&bars->acc_empty[1], 4);
-    mbar_init(&bars->drain, 1);
-    mbar_init(&bars->meta_full[0], 1);
-    mbar_init(&bars->meta_full[1], 1);
-    mbar_init(&bars->gate_full[0], 1);
-    mbar_init(&bars->gate_full[1], 1);
-    bars->abort = 0;
-    bars->is_last = 0;
-    bars->dep_ready = 0;
-    mbar_fence_init();
-  }
   if (warp == kWarpMma) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
     tmem_relinquish();
-  }
-  if (warp == kWarpProducer && lane == 0) {
-    prefetch_tensormap(&tm_x);
-    if (p.tma_out) prefetch_tensormap(&tm_y);
-    if (p.tma_out && p.gate) prefetch_tensormap(&tm_g);
-    if (!kPack) prefetch_tensormap(&tm_wa);
-    if (L != kBF16 && !kPack) prefetch_tensormap(&tm_wb);
   }
   tc_fence_before();
   __syncthreads();
@@ -308,197 +432,226 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 
   if (warp == kWarpProducer) {
     // ------------------------------ producer --------------------------------
-    uint32_t* meta = reinterpret_cast<uint32_t*>(smem + p.meta_off);
-    int meta_issued[2] = {0, 0};
-    // per-m-tile verbatim flags and prefix counts for its 128 rows
-    auto issue_meta = [&](int mt, int slot) {
-      uint32_t* dst = meta + slot * 2 * p.meta_slot_words;
-      const int64_t row0 = static_cast<int64_t>(mt) * 128;
-      const int rows = static_cast<int>(p.N - row0 < 128 ? p.N - row0 : 128);
-      const uint32_t words = static_cast<uint32_t>(rows) * p.wpr;
-      const uint32_t bulk_words = words & ~3u;  // 16-byte multiple
-      if (lane == 0) {
-        const uint32_t tx = bulk_words ? 2 * bulk_words * 4 : 0;
-        mbar_arrive_expect_tx(&bars->meta_full[slot], tx);
-        if (bulk_words) {
-          bulk_load(dst, p.vflags + row0 * p.wpr, bulk_words * 4, &bars->meta_full[slot]);
-          bulk_load(dst + p.meta_slot_words, p.vprefix + row0 * p.wpr, bulk_words * 4, &bars->meta_full[slot]);
-        }
-      }
-      // tail words and rows past the matrix: plain loads / zeros
-      for (uint32_t w = bulk_words + lane; w < p.meta_slot_words; w += 32) {
-        dst[w] = w < words ? p.vflags[row0 * p.wpr + w] : 0u;
-        dst[p.meta_slot_words + w] = w < words ? p.vprefix[row0 * p.wpr + w] : 0u;
-      }
-      __syncwarp();
-      ++meta_issued[slot];
-    };
-    if (kIdx4) {
-      issue_meta(mt_first, 0);
-      if (mt_first + 1 <= mt_last) issue_meta(mt_first + 1, 1);
-    }
-    int cur_mt = -1;
-    int64_t i = 0;
-    const uint64_t stream_policy = l2_evict_first();
     // Activations may be the output of the previous kernel on the stream
     // (programmatic dependent launch lets this kernel start while that one
-    // finishes).  Weight copies of the first S stages go out at once; their
-    // activation tiles, which complete the same barriers, follow as soon as
-    // an epilogue thread has seen that kernel complete (dep_ready), at the
-    // latest after the S-th weight copy.
-    bool dep_done = false;
-    int64_t x_next = 0;  // first-use stages whose activation tile is issued
-    int kbx = static_cast<int>(u0 % p.KB);
-    int ntx = static_cast<int>((u0 / p.KB) % p.n_ntiles);
-    auto finish_dependency = [&](int64_t n_issued) {
-      griddep_wait();  // immediate once dep_ready is set; formal ordering
-      dep_done = true;
-      for (; x_next < n_issued; ++x_next) {  // stage x_next, first use
-        if (lane == 0)
-          tma_load_2d(smem + static_cast<size_t>(x_next) * p.stage_bytes + p.off_x, &tm_x, kbx * 64,
-                      ntx * p.ntile, &bars->full[x_next]);
-        if (++kbx == p.KB) {
-          kbx = 0;
-          if (++ntx == p.n_ntiles) ntx = 0;
+    // finishes).  Weight copies go out at once; activation tiles, which
+    // complete the same barriers, follow as soon as an epilogue thread has
+    // seen that kernel complete (dep_ready), at the latest after the S-th
+    // stage.
+    if constexpr (!kIdx4) {
+      if (lane == 0) {
+        bool dep_done = false;
+        StageWalk w, wx;
+        walk_init(w, u0, u1, p);
+        wx = w;
+        int sx = 0;          // ring slot of the first stage without its activation tile
+        int64_t x_next = 0;  // that stage's index
+        int s = 0;
+        uint32_t k = 0;
+        int64_t st = 0;
+        auto issue_deferred_x = [&](int64_t upto) {
+          for (; x_next < upto; ++x_next) {
+            issue_x(sx, wx);
+            walk_next(wx, u1, p);
+            if (++sx == S) sx = 0;
+          }
+        };
+        for (; w.u < u1; walk_next(w, u1, p), ++st) {
+          if (st > 0 && ++s == S) {
+            s = 0;
+            ++k;
+          }
+          if (k > 0 && !mbar_wait(&bars->empty[s], (k - 1) & 1, &bars->abort, p.status)) break;
+          uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
+          uint32_t tx = static_cast<uint32_t>(p.ks) * p.x_kb_bytes;
+          const bool w_early = st < early;
+          if (!w_early) tx += weight_bytes(w);
+          uint32_t t_first = 0, t_rows = 0;
+          if constexpr (kPack) {
+            // verbatim rows of the stage's tiles: one contiguous run
+            const int64_t slot = static_cast<int64_t>(w.mt) * p.KB + w.kb - pt_min;
+            if (slot >= 0 && slot + w.n < p.n_soff) {
+              const uint32_t a = soff[slot], b = soff[slot + w.n];
+              if (b < a || b - a > 128u * static_cast<uint32_t>(w.n) || static_cast<long long>(b) > p.n_verbatim) {
+                record_status(p.status, UW_ERR_CORRUPT);
+              } else {
+                t_first = a;
+                t_rows = b - a < static_cast<uint32_t>(p.vcap) ? b - a : static_cast<uint32_t>(p.vcap);
+              }
+            } else {
+              record_status(p.status, UW_ERR_CORRUPT);
+            }
+            tx += t_rows * 128u;
+          }
+          mbar_arrive_expect_tx(&bars->full[s], tx);
+          if (!w_early) issue_weights(s, w);
+          if (kPack && t_rows)
+            bulk_load_hint(stage + p.off_verb, p.tails + static_cast<uint64_t>(t_first) * 128u, t_rows * 128u,
+                           &bars->full[s], stream_policy);
+          if (dep_done) {
+            issue_x(s, w);
+          } else if (ld_acquire_cta(&bars->dep_ready) || st == S - 1 || w.u + w.n >= u1) {
+            griddep_wait();  // immediate once dep_ready is set; formal ordering
+            dep_done = true;
+            issue_deferred_x(st + 1);
+          }
         }
+        // stopped early (an abort): stages whose weights went out before the
+        // tables arrived still need their arrive; the previous kernel must be
+        // waited for and the issued stages' activation tiles completed
+        if (!dep_done) {
+          griddep_wait();
+          issue_deferred_x(st);
+        }
+        for (int64_t e = st; e < early; ++e) mbar_arrive(&bars->full[e]);
+        // drain: the last use of every stage must land before the CTA exits
+        // (normally already complete)
+        const int64_t issued = st > early ? st : early;
+        for (int64_t q = issued - S > 0 ? issued - S : 0; q < issued; ++q)
+          mbar_wait(&bars->full[q % S], static_cast<uint32_t>(q / S) & 1, nullptr, p.status);
       }
       __syncwarp();
-    };
-    // the loop advances (stage, use) and (row block, batch tile, k-block)
-    // incrementally: no division per unit
-    int s = 0;
-    uint32_t k = 0;
-    int kb, mt, nt;
-    {
-      const int64_t t0 = u0 / p.KB;
-      kb = static_cast<int>(u0 - t0 * p.KB);
-      mt = static_cast<int>(t0 / p.n_ntiles);
-      nt = static_cast<int>(t0 - static_cast<int64_t>(mt) * p.n_ntiles);
-    }
-    for (int64_t u = u0; u < u1; ++u, ++i) {
-      if (i > 0) {
-        if (++s == S) {
+    } else {
+      // run-time transcode (one k-block per stage): the warp stages each row
+      // tile's verbatim flags and prefix counts, finds the verbatim rows of
+      // every k-block with one ballot per 32 rows and copies up to kVCap of
+      // them next to the tile
+      uint32_t* meta = reinterpret_cast<uint32_t*>(smem + p.meta_off);
+      int meta_issued[2] = {0, 0};
+      auto issue_meta = [&](int mt, int slot) {
+        uint32_t* dst = meta + slot * 2 * p.meta_slot_words;
+        const int64_t row0 = static_cast<int64_t>(mt) * 128;
+        const int rows = static_cast<int>(p.N - row0 < 128 ? p.N - row0 : 128);
+        const uint32_t words = static_cast<uint32_t>(rows) * p.wpr;
+        const uint32_t bulk_words = words & ~3u;  // 16-byte multiple
+        if (lane == 0) {
+          const uint32_t tx = bulk_words ? 2 * bulk_words * 4 : 0;
+          mbar_arrive_expect_tx(&bars->meta_full[slot], tx);
+          if (bulk_words) {
+            bulk_load(dst, p.vflags + row0 * p.wpr, bulk_words * 4, &bars->meta_full[slot]);
+            bulk_load(dst + p.meta_slot_words, p.vprefix + row0 * p.wpr, bulk_words * 4, &bars->meta_full[slot]);
+          }
+        }
+        // tail words and rows past the matrix: plain loads / zeros
+        for (uint32_t w = bulk_words + lane; w < p.meta_slot_words; w += 32) {
+          dst[w] = w < words ? p.vflags[row0 * p.wpr + w] : 0u;
+          dst[p.meta_slot_words + w] = w < words ? p.vprefix[row0 * p.wpr + w] : 0u;
+        }
+        __syncwarp();
+        ++meta_issued[slot];
+      };
+      issue_meta(mt_first, 0);
+      if (mt_first + 1 <= mt_last) issue_meta(mt_first + 1, 1);
+      int cur_mt = -1;
+      bool dep_done = false;
+      StageWalk w, wx;
+      walk_init(w, u0, u1, p);
+      wx = w;
+      int sx = 0;
+      int64_t x_next = 0;
+      int s = 0;
+      uint32_t k = 0;
+      int64_t st = 0;
+      auto finish_dependency = [&](int64_t upto) {
+        griddep_wait();
+        dep_done = true;
+        for (; x_next < upto; ++x_next) {
+          if (lane == 0) issue_x(sx, wx);
+          walk_next(wx, u1, p);
+          if (++sx == S) sx = 0;
+        }
+        __syncwarp();
+      };
+      for (; w.u < u1; walk_next(w, u1, p), ++st) {
+        if (st > 0 && ++s == S) {
           s = 0;
           ++k;
         }
-        if (++kb == p.KB) {
-          kb = 0;
-          if (++nt == p.n_ntiles) {
-            nt = 0;
-            ++mt;
-          }
+        if (k > 0 && !warp_wait(&bars->empty[s], (k - 1) & 1, bars, p.status)) break;
+        uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
+        uint32_t tx = static_cast<uint32_t>(p.ks) * p.x_kb_bytes + weight_bytes(w);
+        const int jm = w.mt - mt_first;
+        if (w.mt != cur_mt) {
+          if (jm >= 1 && w.mt + 1 <= mt_last) issue_meta(w.mt + 1, (jm + 1) & 1);
+          if (!warp_wait(&bars->meta_full[jm & 1], (jm >> 1) & 1, bars, p.status)) break;
+          cur_mt = w.mt;
         }
-      }
-      if (k > 0 && !warp_wait(&bars->empty[s], (k - 1) & 1, bars, p.status)) break;
-      uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
-      uint32_t tx = p.x_bytes + p.wa_bytes + p.wb_bytes;
-      uint32_t rec_o0 = 0, rec_bytes = 0;
-      if (kPack) {
-        const int64_t slot = static_cast<int64_t>(mt) * p.KB + kb - pt_min;
-        if (slot + 1 < p.n_soff) {
-          rec_o0 = soff[slot];
-          rec_bytes = (soff[slot + 1] - rec_o0) * 16u;
-        }
-        if (rec_bytes < kRecVerb || rec_bytes > kRecMax || ((rec_bytes - kRecVerb) & 127)) {
-          // inconsistent offsets: load nothing for this tile (bounded garbage)
-          if (lane == 0) record_status(p.status, UW_ERR_CORRUPT);
-          rec_bytes = 0;
-        }
-        // verbatim rows past the staged ones are read from HBM by the rebuild
-        if (rec_bytes > kRecVerb + p.vcap * 128u) rec_bytes = kRecVerb + p.vcap * 128u;
-        tx = p.x_bytes + rec_bytes;
-      }
-      int vq_dst[4];
-      int64_t vq_src[4];
-      if (kIdx4) {
-        const int j = mt - mt_first;
-        if (mt != cur_mt) {
-          if (j >= 1 && mt + 1 <= mt_last) issue_meta(mt + 1, (j + 1) & 1);
-          if (!warp_wait(&bars->meta_full[j & 1], (j >> 1) & 1, bars, p.status)) break;
-          cur_mt = mt;
-        }
-        const uint32_t* mf = meta + (j & 1) * 2 * p.meta_slot_words;
+        const uint32_t* mf = meta + (jm & 1) * 2 * p.meta_slot_words;
         const uint32_t* mp = mf + p.meta_slot_words;
-        const int fwi = kb >> 5;
-        const uint32_t fbit = 1u << (kb & 31);
+        const int fwi = w.kb >> 5;
+        const uint32_t fbit = 1u << (w.kb & 31);
         uint32_t* hdr = reinterpret_cast<uint32_t*>(stage + p.off_hdr);
-        int total = 0;
+        int total = 0, n_copy = 0;
+        int vq_dst[4];
+        int64_t vq_src[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int r = q * 32 + lane;
-          const uint32_t w = mf[r * p.wpr + fwi];
-          const bool v = (w & fbit) != 0;
+          const uint32_t fw = mf[r * p.wpr + fwi];
+          const bool v = (fw & fbit) != 0;
           const uint32_t m = __ballot_sync(0xFFFFFFFFu, v);
           const int idx = total + __popc(m & ((1u << lane) - 1));
-          vq_dst[q] = (v && idx < kVCap) ? idx : -1;
-          vq_src[q] = static_cast<int64_t>(mp[r * p.wpr + fwi]) + __popc(w & (fbit - 1));
+          vq_src[q] = static_cast<int64_t>(mp[r * p.wpr + fwi]) + __popc(fw & (fbit - 1));
+          // a slot outside the store (corrupt flags or prefixes) is not
+          // copied; that row is rebuilt from stale data, bounded
+          const bool in_store = vq_src[q] < p.n_verbatim;
+          if (v && !in_store) record_status(p.status, UW_ERR_CORRUPT);
+          vq_dst[q] = (v && idx < kVCap && in_store) ? idx : -1;
           if (lane == 0) hdr[q] = m;
           total += __popc(m);
+          n_copy += __popc(__ballot_sync(0xFFFFFFFFu, vq_dst[q] >= 0));
         }
-        tx += static_cast<uint32_t>(min(total, kVCap)) * 128u;
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&bars->full[s], tx);
-        if (dep_done) tma_load_2d(stage + p.off_x, &tm_x, kb * 64, nt * p.ntile, &bars->full[s]);
-        if (kPack) {
-          if (rec_bytes)
-            bulk_load_hint(stage + p.off_rec, p.pack + static_cast<uint64_t>(rec_o0) * 16, rec_bytes, &bars->full[s],
-                           stream_policy);
-        } else if (L == kIDX4U || L == kIDX4M) {
-          tma_load_2d(stage + p.off_wa, &tm_wa, kb * 64, mt * 128, &bars->full[s]);
-          tma_load_2d(stage + p.off_wb, &tm_wb, kb * 32, mt * 128, &bars->full[s]);
-        } else if (L == kEXP8) {
-          tma_load_2d(stage + p.off_wa, &tm_wa, kb * 64, mt * 128, &bars->full[s]);
-          tma_load_2d(stage + p.off_wb, &tm_wb, kb * 64, mt * 128, &bars->full[s]);
-        } else {
-          tma_load_2d(stage + p.off_wa, &tm_wa, kb * 64, mt * 128, &bars->full[s]);
+        tx += static_cast<uint32_t>(n_copy) * 128u;
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&bars->full[s], tx);
+          issue_weights(s, w);
+          if (dep_done) issue_x(s, w);
         }
-      }
-      __syncwarp();
-      if (kIdx4) {
+        __syncwarp();
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           if (vq_dst[q] >= 0)
             bulk_load(stage + p.off_verb + vq_dst[q] * 128, p.verbatim + vq_src[q] * 64, 128, &bars->full[s]);
+        if (!dep_done) {
+          const uint32_t ready = __shfl_sync(0xFFFFFFFFu, lane == 0 ? ld_acquire_cta(&bars->dep_ready) : 0u, 0);
+          if (ready || st == S - 1 || w.u + w.n >= u1) finish_dependency(st + 1);
+        }
       }
-      if (!dep_done) {
-        const uint32_t ready = __shfl_sync(0xFFFFFFFFu, lane == 0 ? ld_acquire_cta(&bars->dep_ready) : 0u, 0);
-        if (ready || i == S - 1 || u == u1 - 1) finish_dependency(i + 1);
+      if (!dep_done) finish_dependency(st);
+      if (lane == 0) {
+        for (int64_t q = st - S > 0 ? st - S : 0; q < st; ++q)
+          mbar_wait(&bars->full[q % S], static_cast<uint32_t>(q / S) & 1, nullptr, p.status);
+        for (int sl = 0; sl < 2; ++sl)
+          if (meta_issued[sl] > 0) mbar_wait(&bars->meta_full[sl], (meta_issued[sl] - 1) & 1, nullptr, p.status);
       }
-    }
-    // stopped before the first S stages were issued (an abort): still wait
-    // for the previous kernel, and complete the issued stages' barriers
-    if (!dep_done) finish_dependency(i);
-    // drain: the last use of every stage and every issued flag load must land
-    // before the CTA can exit (normally already complete)
-    if (lane == 0) {
-      const int64_t issued = i;
-      for (int64_t q = issued - S > 0 ? issued - S : 0; q < issued; ++q)
-        mbar_wait(&bars->full[q % S], static_cast<uint32_t>(q / S) & 1, nullptr, p.status);
-      for (int sl = 0; sl < 2; ++sl)
-        if (meta_issued[sl] > 0) mbar_wait(&bars->meta_full[sl], (meta_issued[sl] - 1) & 1, nullptr, p.status);
+      __syncwarp();
     }
   } else if (warp == kWarpMma) {
     // ----------------------------- MMA issuer -------------------------------
-    // One thread issues every MMA (one thread issues an M=128, K=16
-    // tcgen05.mma about every 50 cycles at N <= 64, so a 64-column stage costs
-    // ~0.1 us of issue plus its two barrier waits and commit).  The loop
-    // carries all indices incrementally and does nothing but wait, issue and
-    // commit.
+    // One thread issues every MMA: per stage it waits for the stage's copies
+    // and its rebuilt A tiles, issues 4 MMAs (K = 16 each) per k-block and
+    // commits once.
     if (lane == 0) {
+      StageWalk w;
+      walk_init(w, u0, u1, p);
       int s = 0;
       uint32_t k = 0;
-      int kb = static_cast<int>(u0 % p.KB);
-      uint32_t ab = 0;                    // accumulator buffer of this segment
-      uint32_t use_par[2] = {0u, 0u};     // completed-drain parity per buffer
-      uint32_t used[2] = {0u, 0u};        // segments already run per buffer
+      int64_t st = 0;
+      uint32_t ab = 0;                 // accumulator buffer of this segment
+      uint32_t use_par[2] = {0u, 0u};  // completed-drain parity per buffer
+      uint32_t used[2] = {0u, 0u};     // segments already run per buffer
       const uint32_t acc_stride = static_cast<uint32_t>(p.ntile);
       const uint64_t b_desc0 = smem_desc_sw128(smem_u32(smem + p.off_x));
       const uint64_t b_step = static_cast<uint64_t>(p.stage_bytes >> 4);
+      const uint64_t b_kb = static_cast<uint64_t>(p.x_kb_bytes >> 4);
       bool first = true;
-      for (int64_t u = u0; u < u1; ++u) {
-        const bool last = (u == u1 - 1) || kb == p.KB - 1;
+      for (; w.u < u1; walk_next(w, u1, p), ++st) {
+        if (st > 0 && ++s == S) {
+          s = 0;
+          ++k;
+        }
+        const bool last = (w.u + w.n == u1) || (w.kb + w.n == p.KB);
         const uint32_t d_tmem = tmem + kAccCol + ab * acc_stride;
         if (first && used[ab] > 0) {
           if (!mbar_wait(&bars->acc_empty[ab], use_par[ab], &bars->abort, p.status)) break;
@@ -508,12 +661,16 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         if (!mbar_wait(&bars->full[s], k & 1, &bars->abort, p.status)) break;
         if (!mbar_wait(&bars->rebuilt[s], k & 1, &bars->abort, p.status)) break;
         tc_fence_after();
-        const uint32_t a_tmem = tmem + p.a_col0 + static_cast<uint32_t>(s) * 32;
+        const uint32_t a_tmem = tmem + p.a_col0 + static_cast<uint32_t>(s * p.ks) * 32;
         const uint64_t b_desc = b_desc0 + static_cast<uint64_t>(s) * b_step;
-        mma_ts(d_tmem, a_tmem + 0, b_desc + 0, p.idesc, first ? 0u : 1u);
-        mma_ts(d_tmem, a_tmem + 8, b_desc + 2, p.idesc, 1u);
-        mma_ts(d_tmem, a_tmem + 16, b_desc + 4, p.idesc, 1u);
-        mma_ts(d_tmem, a_tmem + 24, b_desc + 6, p.idesc, 1u);
+        for (int j = 0; j < w.n; ++j) {
+          const uint32_t a = a_tmem + static_cast<uint32_t>(j) * 32;
+          const uint64_t b = b_desc + static_cast<uint64_t>(j) * b_kb;
+          mma_ts(d_tmem, a + 0, b + 0, p.idesc, (first && j == 0) ? 0u : 1u);
+          mma_ts(d_tmem, a + 8, b + 2, p.idesc, 1u);
+          mma_ts(d_tmem, a + 16, b + 4, p.idesc, 1u);
+          mma_ts(d_tmem, a + 24, b + 6, p.idesc, 1u);
+        }
         tc_commit(&bars->empty[s]);
         if (last) {
           tc_commit(&bars->acc_full[ab]);
@@ -521,11 +678,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           if (p.n_acc == 2) ab ^= 1u;
         }
         first = last;
-        if (++s == S) {
-          s = 0;
-          ++k;
-        }
-        if (++kb == p.KB) kb = 0;
       }
       // every MMA issued so far must finish before tensor memory is freed
       tc_commit(&bars->drain);
@@ -537,56 +689,71 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const int grp = (warp - kWarpRebuild0) >> 2;
-    int s = grp;  // group g takes units u0+g, u0+g+G, ... (G <= S)
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + p.a_col0;
+    StageWalk w;
+    walk_init(w, u0, u1, p);
+    int s = 0;
     uint32_t k = 0;
-    while (s >= S) {
-      s -= S;
-      ++k;
-    }
-    for (int64_t u = u0 + grp; u < u1; u += G) {
-      if (u != u0 + grp) {
-        s += G;
-        if (s >= S) {
-          s -= S;
+    int turn = 0;  // stage index modulo G
+    for (int64_t st = 0; w.u < u1; walk_next(w, u1, p), ++st) {
+      if (st > 0) {
+        if (++s == S) {
+          s = 0;
           ++k;
         }
+        if (++turn == G) turn = 0;
       }
+      if (turn != grp) continue;
       if (!warp_wait(&bars->full[s], k & 1, bars, p.status)) break;
       tc_fence_after();
       const uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
-      uint32_t o[32];
-      rebuild_row<L>(stage, p, r, o);
-      if (kIdx4 || kPack) {
-        // verbatim rows: one flag bit per row and k-block, no per-element test
-        const uint32_t* hdr = reinterpret_cast<const uint32_t*>(stage + p.off_hdr);
-        const uint32_t m = hdr[q];
-        if ((m >> lane) & 1) {
-          int idx = __popc(m & ((1u << lane) - 1));
-          for (int qq = 0; qq < q; ++qq) idx += __popc(hdr[qq]);
-          const uint4* src;
-          if (idx < p.vcap) {
-            src = reinterpret_cast<const uint4*>(stage + p.off_verb + idx * 128);
-          } else {
-            // more verbatim rows than staged slots: read this one from HBM
-            const int64_t t = u / p.KB;
-            const int kb = static_cast<int>(u - t * p.KB);
-            const int64_t n = (t / p.n_ntiles) * 128 + r;
-            const int64_t fw = n * p.wpr + (kb >> 5);
-            const uint32_t fl = p.vflags[fw];
-            const int64_t slot = static_cast<int64_t>(p.vprefix[fw]) + __popc(fl & ((1u << (kb & 31)) - 1));
-            src = reinterpret_cast<const uint4*>(p.verbatim + slot * 64);
+      int vbase = 0;  // pack: verbatim rows of the stage's earlier k-blocks
+#pragma unroll 1
+      for (int j = 0; j < w.n; ++j) {
+        uint32_t o[32];
+        rebuild_row<L>(stage, p, r, j, o);
+        if constexpr (kPack) {
+          // verbatim rows: one mask bit per row and k-block, no per-element test
+          const uint4 mk = lds128(stage + p.off_wa + j * kBody + kBodyMask);
+          const uint32_t m = mask_word(mk, q);
+          if ((m >> lane) & 1) {
+            const int idx = vbase + mask_below(mk, q) + __popc(m & ((1u << lane) - 1));
+            if (idx < p.vcap) {
+              copy_row(reinterpret_cast<const uint4*>(stage + p.off_verb + idx * 128), o);
+            } else {
+              // more verbatim rows than staged ones: this one from HBM
+              const int64_t slot = static_cast<int64_t>(w.mt) * p.KB + w.kb - pt_min;
+              const long long g = static_cast<long long>(soff[slot]) + idx;
+              if (g < p.n_verbatim)
+                copy_row(reinterpret_cast<const uint4*>(p.tails + static_cast<uint64_t>(g) * 128u), o);
+              else
+                record_status(p.status, UW_ERR_CORRUPT);
+            }
           }
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint4 v = src[j];
-            o[4 * j] = v.x;
-            o[4 * j + 1] = v.y;
-            o[4 * j + 2] = v.z;
-            o[4 * j + 3] = v.w;
+          vbase += __popc(mk.x) + __popc(mk.y) + __popc(mk.z) + __popc(mk.w);
+        } else if constexpr (kIdx4) {
+          const uint32_t* hdr = reinterpret_cast<const uint32_t*>(stage + p.off_hdr);
+          const uint32_t m = hdr[q];
+          if ((m >> lane) & 1) {
+            int idx = __popc(m & ((1u << lane) - 1));
+            for (int qq = 0; qq < q; ++qq) idx += __popc(hdr[qq]);
+            if (idx < p.vcap) {
+              copy_row(reinterpret_cast<const uint4*>(stage + p.off_verb + idx * 128), o);
+            } else {
+              // more verbatim rows than staged slots: read this one from HBM
+              const int64_t n = static_cast<int64_t>(w.mt) * 128 + r;
+              const int64_t fw = n * p.wpr + (w.kb >> 5);
+              const uint32_t fl = p.vflags[fw];
+              const int64_t slot = static_cast<int64_t>(p.vprefix[fw]) + __popc(fl & ((1u << (w.kb & 31)) - 1));
+              if (slot < p.n_verbatim)
+                copy_row(reinterpret_cast<const uint4*>(p.verbatim + slot * 64), o);
+              else
+                record_status(p.status, UW_ERR_CORRUPT);
+            }
           }
         }
+        tmem_st32(lane_base + static_cast<uint32_t>(s * p.ks + j) * 32, o);
       }
-      tmem_st32(tmem + (static_cast<uint32_t>(q * 32) << 16) + p.a_col0 + static_cast<uint32_t>(s) * 32, o);
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -612,7 +779,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     __nv_bfloat16* out_s = reinterpret_cast<__nv_bfloat16*>(smem + p.epi_off);
     __nv_bfloat16* gate_s = out_s + 2 * 16 * 128;
     const bool tma_gate = p.tma_out && p.gate != nullptr;
-    uint32_t ch = 0;        // output chunks of this CTA so far (buffer ch & 1)
+    uint32_t ch = 0;         // output chunks of this CTA so far (buffer ch & 1)
     uint32_t gate_next = 0;  // gate chunks issued (elected thread)
     auto load_gate = [&](uint32_t chunk, int mt_, int b0) {
       gate_next = chunk + 1;
@@ -787,9 +954,9 @@ __global__ void swiglu_kernel(const __nv_bfloat16* __restrict__ g, const __nv_bf
 // ------------------------------ host side ------------------------------------
 
 struct Layout {
-  int stages = 0;
-  uint32_t stage_bytes = 0, off_x = 0, off_wa = 0, off_wb = 0, off_verb = 0, off_hdr = 0, off_rec = 0;
-  uint32_t x_bytes = 0, wa_bytes = 0, wb_bytes = 0;
+  int stages = 0, ks = 1;
+  uint32_t stage_bytes = 0, off_x = 0, off_wa = 0, off_wb = 0, off_verb = 0, off_hdr = 0;
+  uint32_t x_kb_bytes = 0;
   uint32_t meta_off = 0, meta_slot_words = 0, bar_off = 0, soff_off = 0, a_col0 = 0, epi_off = 0;
   int n_soff = 0, vcap = 0;
   size_t smem = 0;
@@ -797,61 +964,74 @@ struct Layout {
 
 uint32_t a1024(uint32_t v) { return (v + 1023u) & ~1023u; }
 
+int env_int(const char* name, int dflt, int lo, int hi) {
+  const char* e = std::getenv(name);
+  int x = e ? std::atoi(e) : dflt;
+  return x < lo ? lo : (x > hi ? hi : x);
+}
+
 // Pipeline depth cap (UW_MAX_STAGES overrides, for tuning).
 int max_stages() {
-  static int v = [] {
-    const char* e = std::getenv("UW_MAX_STAGES");
-    int x = e ? std::atoi(e) : kMaxStages;
-    return x < 2 ? 2 : (x > kMaxStages ? kMaxStages : x);
-  }();
+  static int v = env_int("UW_MAX_STAGES", kMaxStages, 2, kMaxStages);
   return v;
 }
 
 // Rebuild warpgroups per CTA (UW_REBUILD_GROUPS overrides, for tuning).
 int rebuild_groups() {
-  static int g = [] {
-    const char* e = std::getenv("UW_REBUILD_GROUPS");
-    int v = e ? std::atoi(e) : 2;
-    return v < 1 ? 1 : (v > kMaxGroups ? kMaxGroups : v);
-  }();
+  static int g = env_int("UW_REBUILD_GROUPS", 2, 1, kMaxGroups);
   return g;
+}
+
+// k-blocks per stage: several for small batch tiles, where the per-stage
+// costs dominate; one when the activation tile is large (UW_STAGE_KBLOCKS
+// overrides, for tuning).
+int stage_kblocks(int loader, int ntile, int KB) {
+  static int forced = env_int("UW_STAGE_KBLOCKS", 0, 0, kMaxKS);
+  int ks;
+  if (loader_idx4(loader)) ks = 1;
+  else if (forced) ks = forced;
+  else if (loader == kBF16) ks = ntile <= 32 ? 2 : 1;
+  else ks = ntile <= 64 ? 2 : 1;
+  return std::max(1, std::min(ks, KB));
 }
 
 // Shared-memory plan of one launch.  Every tile region starts on a 1024-byte
 // boundary (the 128-byte swizzle of the activation tile repeats every 1024).
 bool make_layout(int loader, const GemmPlan& plan, int wpr, bool tma_out, bool gate, Layout* out) {
   Layout l;
-  // TMEM: accumulators (n_acc x ntile columns), then one 32-column A tile per
-  // stage
+  l.ks = stage_kblocks(loader, plan.ntile, plan.KB);
+  const uint32_t ks = static_cast<uint32_t>(l.ks);
+  // TMEM: accumulators (n_acc x ntile columns), then 32 columns of rebuilt A
+  // per k-block of every stage
   const int n_acc = 2 * plan.ntile <= 256 ? 2 : 1;
   l.a_col0 = (static_cast<uint32_t>(n_acc * plan.ntile) + 31u) & ~31u;
-  const int tmem_stages = static_cast<int>((kTmemCols - l.a_col0) / 32u);
-  l.x_bytes = static_cast<uint32_t>(plan.ntile) * 128;
-  const bool idx4 = loader == kIDX4U || loader == kIDX4M;
+  const int tmem_stages = static_cast<int>((kTmemCols - l.a_col0) / (32u * ks));
+  l.x_kb_bytes = static_cast<uint32_t>(plan.ntile) * 128;
+  const bool idx4 = loader_idx4(loader);
   const bool pack = loader_pack(loader);
   l.off_x = 0;
+  l.off_wa = a1024(ks * l.x_kb_bytes);
   if (pack) {
-    l.off_rec = a1024(l.x_bytes);
-    l.off_wa = l.off_rec;
-    l.off_wb = l.off_rec + kRecIdx;
-    l.off_hdr = l.off_rec + kRecMask;
-    l.off_verb = l.off_rec + kRecVerb;
-    l.vcap = kRecVCap;  // final value below, from the stage count
-    l.stage_bytes = a1024(l.off_rec + kRecVerb + kPackMinVCap * 128u);
+    l.off_wb = l.off_wa + kBodyIdx;  // unused: indices are inside each body
+    l.off_verb = (l.off_wa + ks * kBody + 127u) & ~127u;
+    l.stage_bytes = a1024(l.off_verb + kPackMinTail * 128u);
+  } else if (loader == kBF16) {
+    l.off_wb = l.off_wa;
+    l.stage_bytes = l.off_wa + ks * 16384u;
+  } else if (loader == kEXP8) {
+    l.off_wb = l.off_wa + ks * 8192u;
+    l.stage_bytes = l.off_wb + ks * 8192u;
   } else {
-    l.wa_bytes = loader == kBF16 ? 16384u : 8192u;
-    l.wb_bytes = loader == kBF16 ? 0u : (loader == kEXP8 ? 8192u : 4096u);
-    l.off_wa = a1024(l.off_x + l.x_bytes);
-    l.off_wb = a1024(l.off_wa + l.wa_bytes);
-    l.off_verb = a1024(l.off_wb + l.wb_bytes);
-    l.off_hdr = l.off_verb + (idx4 ? kVCap * 128u : 0u);
+    l.off_wb = l.off_wa + ks * 8192u;
+    l.off_verb = a1024(l.off_wb + ks * 4096u);
+    l.off_hdr = l.off_verb + kVCap * 128u;
     l.vcap = kVCap;
-    l.stage_bytes = a1024(l.off_hdr + (idx4 ? 64u : 0u));
+    l.stage_bytes = a1024(l.off_hdr + 64u);
   }
   l.meta_slot_words = idx4 ? 128u * static_cast<uint32_t>(wpr) : 0u;
   const uint32_t meta_bytes = a1024(2u * 2u * l.meta_slot_words * 4u);
-  // pack: record offsets of every tile one CTA can reach (its units span at
-  // most `span` row blocks)
+  // pack: verbatim-row offsets of every tile one CTA can reach (its units
+  // span at most `span` row blocks)
   if (pack) {
     const int64_t per_cta = (plan.units + plan.grid - 1) / plan.grid;
     const int64_t per_mt = static_cast<int64_t>(plan.KB) * plan.n_ntiles;
@@ -868,12 +1048,12 @@ bool make_layout(int loader, const GemmPlan& plan, int wpr, bool tma_out, bool g
   if (stages < 2) return false;
   l.stages = stages;
   if (pack) {
-    // pack records: spread the remaining shared memory over the stages as
-    // on-chip verbatim rows (most tiles have a few; the rest come from HBM)
+    // spread the remaining shared memory over the stages as on-chip verbatim
+    // rows (most tiles have a few; the rest come from HBM)
     const uint32_t per_stage = ((kSmemLimit - fixed) / static_cast<uint32_t>(stages)) & ~1023u;
-    const uint32_t room = (per_stage - l.off_rec - kRecVerb) / 128u;
-    l.vcap = static_cast<int>(std::min<uint32_t>(room, kRecVCap));
-    l.stage_bytes = a1024(l.off_rec + kRecVerb + static_cast<uint32_t>(l.vcap) * 128u);
+    const uint32_t room = (per_stage - l.off_verb) / 128u;
+    l.vcap = static_cast<int>(std::min<uint32_t>(room, 128u * ks));
+    l.stage_bytes = a1024(l.off_verb + static_cast<uint32_t>(l.vcap) * 128u);
   }
   l.meta_off = static_cast<uint32_t>(stages) * l.stage_bytes;
   l.soff_off = l.meta_off + meta_bytes;
@@ -960,9 +1140,8 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
     if (!a.sm || !a.aux || !aligned16(a.sm) || !aligned16(a.aux)) return UW_ERR_INVALID_ARG;
     kl = kEXP8;
   } else if (a.loader == kLoaderPACK) {
-    if (!a.pack || !a.pack_off || !a.vflags || !a.vprefix || !a.palette) return UW_ERR_INVALID_ARG;
-    if (!aligned16(a.pack) || !aligned16(a.vflags) || !aligned16(a.vprefix) || (a.verbatim && !aligned16(a.verbatim)))
-      return UW_ERR_INVALID_ARG;
+    if (!a.pack || !a.pack_off || !a.palette) return UW_ERR_INVALID_ARG;
+    if (!aligned16(a.pack) || !aligned16(a.pack_off)) return UW_ERR_INVALID_ARG;
     bool mixed = false;
     pal = palette_tables(a.palette, a.code_len, &mixed);
     kl = (mixed || a.force_mixed_palette) ? kPACKM : kPACKU;
@@ -993,11 +1172,18 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
                                            16, CU_TENSOR_MAP_SWIZZLE_NONE)) != UW_OK)
       return st;
   }
-  if ((st = make_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, a.K, a.B, a.K * 2, 64, plan.ntile,
-                               CU_TENSOR_MAP_SWIZZLE_128B)) != UW_OK)
+  // activations: a stage's ks tiles of [ntile rows x 64 columns] in one 3-D
+  // load (dims: 64 columns, batch rows, k-blocks), else one 2-D load each
+  int x3d = 0;
+  if (lay.ks > 1 &&
+      make_tensor_map_3d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, 64, a.B, a.K / 64, a.K * 2, 128, 64, plan.ntile,
+                         lay.ks, CU_TENSOR_MAP_SWIZZLE_128B) == UW_OK)
+    x3d = 1;
+  if (!x3d && (st = make_tensor_map_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.x, a.K, a.B, a.K * 2, 64,
+                                       plan.ntile, CU_TENSOR_MAP_SWIZZLE_128B)) != UW_OK)
     return st;
   if (loader_pack(kl)) {
-    twa = tx;  // unused: pack records arrive by bulk copy
+    twa = tx;  // unused: pack bodies arrive by bulk copy
     twb = tx;
   } else if (kl == kBF16) {
     if ((st = make_tensor_map_2d(&twa, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.wbf16, a.K, a.N, a.K * 2, 64, 128,
@@ -1028,15 +1214,14 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.units = plan.units;
   kp.grid = plan.grid;
   kp.stages = lay.stages;
+  kp.ks = lay.ks;
   kp.stage_bytes = lay.stage_bytes;
   kp.off_x = lay.off_x;
   kp.off_wa = lay.off_wa;
   kp.off_wb = lay.off_wb;
   kp.off_verb = lay.off_verb;
   kp.off_hdr = lay.off_hdr;
-  kp.x_bytes = lay.x_bytes;
-  kp.wa_bytes = lay.wa_bytes;
-  kp.wb_bytes = lay.wb_bytes;
+  kp.x_kb_bytes = lay.x_kb_bytes;
   kp.meta_off = lay.meta_off;
   kp.meta_slot_words = lay.meta_slot_words;
   kp.bar_off = lay.bar_off;
@@ -1044,6 +1229,7 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.vflags = a.vflags;
   kp.vprefix = a.vprefix;
   kp.verbatim = a.verbatim;
+  kp.n_verbatim = a.n_verbatim;
   kp.y = a.y;
   kp.gate = a.gate;
   uint8_t* ws = static_cast<uint8_t*>(a.ws);
@@ -1056,13 +1242,14 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.vcap = lay.vcap;
   kp.n_acc = 2 * plan.ntile <= 256 ? 2 : 1;
   kp.pack = a.pack;
+  kp.tails = a.pack ? a.pack + static_cast<uint64_t>(plan.n_mtiles) * plan.KB * kBody : nullptr;
   kp.pack_off = a.pack_off;
-  kp.off_rec = lay.off_rec;
   kp.soff_off = lay.soff_off;
   kp.n_soff = lay.n_soff;
   kp.a_col0 = lay.a_col0;
   kp.epi_off = lay.epi_off;
   kp.tma_out = tma_out ? 1 : 0;
+  kp.x3d = x3d;
 
   switch (kl) {
     case kBF16: return launch_kernel<kBF16>(tx, twa, twb, ty, tg, kp, lay.smem, s, a.overlap_previous);
@@ -1113,6 +1300,7 @@ uw_status run_pipeline(const uw_matrix* m, int pipeline, const uint16_t* x, int3
   a.ws = ws;
   a.ws_bytes = ws_bytes;
   a.wpr = m->L.words_per_row;
+  a.n_verbatim = m->L.n_verbatim;
   a.force_mixed_palette = force_mixed;
   uint32_t* status = static_cast<uint32_t*>(ws);
   const size_t need = pipeline_scratch_bytes(&m->L, pipeline);
@@ -1136,9 +1324,6 @@ uw_status run_pipeline(const uw_matrix* m, int pipeline, const uint16_t* x, int3
       a.loader = kLoaderPACK;
       a.pack = m->pack;
       a.pack_off = m->pack_off;
-      a.vflags = m->vflags;
-      a.vprefix = m->vprefix;
-      a.verbatim = m->verbatim;
       a.palette = m->cb.palette;
       a.code_len = m->cb.code_len;
       break;

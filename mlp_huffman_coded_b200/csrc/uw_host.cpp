@@ -434,19 +434,19 @@ extern "C" uw_status uw_direct_pack_offsets(const uw_layout* L, const uint32_t* 
   const int64_t wpr = (kb_n + 31) / 32;
   if (L->words_per_row != wpr) return UW_ERR_CORRUPT;
   const int64_t mt_n = (L->rows + 127) / 128;
-  uint64_t pos = 0;  // 16-byte units
+  uint64_t rows_before = 0;  // verbatim rows of the tiles so far
   int64_t t = 0;
   for (int64_t mt = 0; mt < mt_n; ++mt) {
     const int64_t r_end = std::min<int64_t>(L->rows, (mt + 1) * 128);
     for (int64_t kb = 0; kb < kb_n; ++kb, ++t) {
-      int nv = 0;
-      for (int64_t n = mt * 128; n < r_end; ++n) nv += (vflags[n * wpr + kb / 32] >> (kb % 32)) & 1;
-      off[t] = static_cast<uint32_t>(pos);
-      pos += (12416 + 128 * std::min(nv, 32)) / 16;
-      if (pos >= (uint64_t(1) << 32)) return UW_ERR_UNSUPPORTED_SHAPE;
+      off[t] = static_cast<uint32_t>(rows_before);
+      for (int64_t n = mt * 128; n < r_end; ++n) rows_before += (vflags[n * wpr + kb / 32] >> (kb % 32)) & 1;
+      if (rows_before >= (uint64_t(1) << 32)) return UW_ERR_UNSUPPORTED_SHAPE;
     }
   }
-  off[t] = static_cast<uint32_t>(pos);
-  if (pack_bytes) *pack_bytes = pos * 16;
+  off[t] = static_cast<uint32_t>(rows_before);
+  const uint64_t bytes = static_cast<uint64_t>(t) * 12304u + rows_before * 128u;
+  if (bytes > (uint64_t(1) << 36)) return UW_ERR_UNSUPPORTED_SHAPE;
+  if (pack_bytes) *pack_bytes = bytes;
   return UW_OK;
 }

@@ -31,6 +31,11 @@ inline uw_status cuda_status(cudaError_t e) { return e == cudaSuccess ? UW_OK : 
 uw_status make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
                              uint64_t inner, uint64_t outer, uint64_t row_stride_bytes,
                              uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
+// Same, 3-D: dims {d0, d1, d2} (d0 contiguous), byte strides of dims 1 and 2
+// (any order, multiples of 16), box {b0, b1, b2}.
+uw_status make_tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0,
+                             uint64_t d1, uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0,
+                             uint32_t b1, uint32_t b2, CUtensorMapSwizzle swizzle);
 
 // Workspace layout: [0, 256) header (status word at offset 0), then tile
 // counters, split-K partials and the pipeline's intermediate matrix.
@@ -72,8 +77,9 @@ struct GemmArgs {
   const uint32_t* vflags = nullptr;
   const uint32_t* vprefix = nullptr;
   const uint16_t* verbatim = nullptr;
+  long long n_verbatim = 0;            // verbatim groups (bounds the slots read)
   int wpr = 0;
-  const uint8_t* pack = nullptr;      // direct-palette records (PACK loader)
+  const uint8_t* pack = nullptr;      // direct-palette pack: bodies, then verbatim tails (PACK loader)
   const uint32_t* pack_off = nullptr;
   const uint8_t* palette = nullptr;   // 16 entries (IDX4 / PACK loaders)
   const uint8_t* code_len = nullptr;  // which palette entries are in use

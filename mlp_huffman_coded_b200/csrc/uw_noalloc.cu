@@ -77,6 +77,7 @@ extern "C" uw_status uw_gemm_direct_palette_noalloc(const uw_matrix* m, const ui
   a.vflags = m->vflags;
   a.vprefix = m->vprefix;
   a.verbatim = m->verbatim;
+  a.n_verbatim = m->L.n_verbatim;
   a.wpr = m->L.words_per_row;
   a.palette = m->cb.palette;
   a.code_len = m->cb.code_len;

@@ -1,7 +1,8 @@
-// Load-time assembly of the direct-palette pack: one contiguous record per
-// 128 x 64 tile holding the tile's sign+mantissa bytes, 4-bit palette
-// indices, verbatim mask and (up to 32) verbatim rows, in the byte order the
-// reconstructive GEMM reads from shared memory.
+// Load-time assembly of the direct-palette pack: for every 128 x 64 tile a
+// fixed-size body holding the tile's sign+mantissa bytes, 4-bit palette
+// indices and verbatim-row mask, in the byte order the reconstructive GEMM
+// reads from shared memory, and, after all bodies, the verbatim rows of every
+// tile in tile order.
 //
 // Method: Cloudflare, "Unweight: how we compressed an LLM 22% without
 // sacrificing quality", section "Four ways to use compressed weights"
@@ -9,14 +10,15 @@
 // loaded) and section "How the reconstructive matmul works" (the producer
 // stages sign+mantissa bytes, palette indices and the verbatim rows of
 // rare-exponent rows).  Gathering them per tile at load time lets the GEMM
-// fetch each tile with one bulk copy from a sequential stream.
+// fetch consecutive tiles with one bulk copy at an address it computes, and
+// their verbatim rows with a second one.
 #include "uw_device.cuh"
 #include "uw_internal.h"
 
 namespace uw {
 namespace {
 
-constexpr int kRecSm = 0, kRecIdx = 8192, kRecMask = 12288, kRecVerb = 12416, kRecVCap = 32;
+constexpr uint32_t kBody = 12304, kBodySm = 0, kBodyIdx = 8192, kBodyMask = 12288;
 
 struct PackParams {
   const uint8_t* sm;
@@ -24,9 +26,10 @@ struct PackParams {
   const uint32_t* vflags;
   const uint32_t* vprefix;
   const uint16_t* verbatim;
-  const uint32_t* off;
+  const uint32_t* off;  // per tile: verbatim rows of all earlier tiles
   uint8_t* pack;
-  int64_t rows, cols;
+  uint8_t* tails;
+  int64_t rows, cols, n_verbatim;
   int KB, wpr;
 };
 
@@ -39,9 +42,7 @@ __global__ void __launch_bounds__(128) pack_kernel(const PackParams p) {
   const int warp = r >> 5, lane = r & 31;
   const int64_t n = mt * 128 + r;
   const bool valid = n < p.rows;
-  const uint64_t rec_bytes = static_cast<uint64_t>(p.off[t + 1] - p.off[t]) * 16;
-  uint8_t* rec = p.pack + static_cast<uint64_t>(p.off[t]) * 16;
-  const bool fits = rec_bytes >= kRecVerb;
+  uint8_t* body = p.pack + static_cast<uint64_t>(t) * kBody;
 
   uint4 s[4] = {}, x[2] = {};
   uint32_t fl = 0, pre = 0;
@@ -61,22 +62,23 @@ __global__ void __launch_bounds__(128) pack_kernel(const PackParams p) {
   const uint32_t m = __ballot_sync(0xFFFFFFFFu, verb);
   if (lane == 0) masks[warp] = m;
   __syncthreads();
-  if (!fits) return;
 #pragma unroll
   for (int j = 0; j < 4; ++j)
-    *reinterpret_cast<uint4*>(rec + kRecSm + r * 64 + 16 * (j ^ ((r >> 1) & 3))) = s[j];
+    *reinterpret_cast<uint4*>(body + kBodySm + r * 64 + 16 * (j ^ ((r >> 1) & 3))) = s[j];
 #pragma unroll
   for (int j = 0; j < 2; ++j)
-    *reinterpret_cast<uint4*>(rec + kRecIdx + r * 32 + 16 * (j ^ ((r >> 2) & 1))) = x[j];
-  if (r < 4) reinterpret_cast<uint32_t*>(rec + kRecMask)[r] = masks[r];
-  if (r >= 4 && r < 32) reinterpret_cast<uint32_t*>(rec + kRecMask)[r] = 0u;  // pad to 128 bytes
+    *reinterpret_cast<uint4*>(body + kBodyIdx + r * 32 + 16 * (j ^ ((r >> 2) & 1))) = x[j];
+  if (r < 4) reinterpret_cast<uint32_t*>(body + kBodyMask)[r] = masks[r];
   if (verb) {
     int idx = __popc(m & ((1u << lane) - 1));
     for (int q = 0; q < warp; ++q) idx += __popc(masks[q]);
-    if (idx < kRecVCap && kRecVerb + (idx + 1) * 128 <= rec_bytes) {
-      const int64_t slot = static_cast<int64_t>(pre) + __popc(fl & below);
+    const uint64_t row = static_cast<uint64_t>(p.off[t]) + static_cast<uint64_t>(idx);
+    const int64_t slot = static_cast<int64_t>(pre) + __popc(fl & below);
+    // offsets or flags that disagree with each other write nothing outside
+    // this tile's rows of the tail region, and read nothing outside the store
+    if (row < p.off[t + 1] && row < static_cast<uint64_t>(p.n_verbatim) && slot < p.n_verbatim) {
       const uint4* vs = reinterpret_cast<const uint4*>(p.verbatim + slot * 64);
-      uint4* vd = reinterpret_cast<uint4*>(rec + kRecVerb + idx * 128);
+      uint4* vd = reinterpret_cast<uint4*>(p.tails + row * 128u);
 #pragma unroll
       for (int j = 0; j < 8; ++j) vd[j] = __ldg(vs + j);
     }
@@ -109,10 +111,12 @@ extern "C" uw_status uw_pack_direct_palette(const uw_matrix* m, const uint32_t* 
   p.pack = out_pack;
   p.rows = m->L.rows;
   p.cols = m->L.cols;
+  p.n_verbatim = m->L.n_verbatim;
   p.KB = static_cast<int>(m->L.cols / 64);
   p.wpr = m->L.words_per_row;
   const int64_t n_tiles = ((m->L.rows + 127) / 128) * p.KB;
   if (n_tiles > 0x7FFFFFFF) return UW_ERR_UNSUPPORTED_SHAPE;
+  p.tails = out_pack + static_cast<uint64_t>(n_tiles) * kBody;
   pack_kernel<<<static_cast<unsigned>(n_tiles), 128, 0, static_cast<cudaStream_t>(stream)>>>(p);
   note_launch();
   if (cudaError_t e = cudaGetLastError(); e != cudaSuccess) return cuda_status(e);

@@ -50,9 +50,9 @@ uw_status device_info(DeviceInfo* out) {
   return UW_OK;
 }
 
-uw_status make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
-                             uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
-                             uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+static uw_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, const void* base,
+                              const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                              CUtensorMapSwizzle swizzle) {
   std::call_once(g_encode_once, [] {
     void* fn = nullptr;
     cudaDriverEntryPointQueryResult q;
@@ -63,14 +63,29 @@ uw_status make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const 
       cudaGetLastError();
   });
   if (!g_encode) return UW_ERR_CUDA;
-  const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {row_stride_bytes};
-  const cuuint32_t box[2] = {box_inner, box_outer};
-  const cuuint32_t estr[2] = {1, 1};
-  CUresult r = g_encode(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, dtype, rank, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? UW_OK : UW_ERR_CUDA;
+}
+
+uw_status make_tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                             uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner,
+                             uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  return encode_tiled(map, dtype, 2, base, dims, strides, box, swizzle);
+}
+
+uw_status make_tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t d0,
+                             uint64_t d1, uint64_t d2, uint64_t stride1_bytes, uint64_t stride2_bytes, uint32_t b0,
+                             uint32_t b1, uint32_t b2, CUtensorMapSwizzle swizzle) {
+  const cuuint64_t dims[3] = {d0, d1, d2};
+  const cuuint64_t strides[2] = {stride1_bytes, stride2_bytes};
+  const cuuint32_t box[3] = {b0, b1, b2};
+  return encode_tiled(map, dtype, 3, base, dims, strides, box, swizzle);
 }
 
 uw_status check_matrix(const uw_matrix* m) {
@@ -141,19 +156,39 @@ extern "C" size_t uw_workspace_bytes(const uw_layout* L, int32_t pipeline, int32
   return gemm_ws_bytes(p) + pipeline_scratch_bytes(L, pipeline);
 }
 
+// Header words: [0] sticky status, [2..3] the workspace's size as given to
+// uw_workspace_init (so that recovery after a failed call can re-zero it).
 extern "C" uw_status uw_workspace_init(void* ws, size_t bytes, void* stream) {
   if (!ws || bytes < kWsHeader || !aligned16(ws)) return UW_ERR_INVALID_ARG;
-  return cuda_status(cudaMemsetAsync(ws, 0, bytes, static_cast<cudaStream_t>(stream)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, bytes, s) != cudaSuccess) return UW_ERR_CUDA;
+  // the size word goes through a stream-ordered copy from a host value that
+  // must outlive it: wait for it
+  const uint64_t size = bytes;
+  if (cudaMemcpyAsync(static_cast<uint8_t*>(ws) + 8, &size, 8, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return UW_ERR_CUDA;
+  return cuda_status(cudaStreamSynchronize(s));
 }
 
 extern "C" uw_status uw_workspace_status(void* ws, void* stream) {
   if (!ws) return UW_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  uint32_t v = 0;
-  if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return UW_ERR_CUDA;
+  uint64_t hdr[2] = {0, 0};
+  if (cudaMemcpyAsync(hdr, ws, 16, cudaMemcpyDeviceToHost, s) != cudaSuccess) return UW_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return UW_ERR_CUDA;
+  const uint32_t v = static_cast<uint32_t>(hdr[0]);
   if (v != 0) {
-    if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return UW_ERR_CUDA;
+    // A call that gave up (a timed-out wait, corrupt data) may have left
+    // split-K tile counters raised; the next call would then read partial
+    // sums nobody wrote.  Re-zero the whole workspace (its size is in the
+    // header when uw_workspace_init set it up), keeping that size word.
+    const uint64_t size = hdr[1];
+    if (size >= kWsHeader) {
+      if (cudaMemsetAsync(ws, 0, 8, s) != cudaSuccess) return UW_ERR_CUDA;
+      if (cudaMemsetAsync(static_cast<uint8_t*>(ws) + 16, 0, size - 16, s) != cudaSuccess) return UW_ERR_CUDA;
+    } else if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) {
+      return UW_ERR_CUDA;
+    }
     if (cudaStreamSynchronize(s) != cudaSuccess) return UW_ERR_CUDA;
   }
   return static_cast<uw_status>(v);

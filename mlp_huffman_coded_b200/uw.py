@@ -229,7 +229,9 @@ class Workspace:
     def __init__(self, nbytes: int, device="cuda"):
         import torch
         self.nbytes = max(int(nbytes), 256)
-        self.t = torch.zeros(self.nbytes, dtype=torch.uint8, device=device)
+        self.t = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        with torch.cuda.device(self.t.device):
+            _check(lib().uw_workspace_init(self.ptr, self.nbytes, _stream(None)), "uw_workspace_init")
 
     @property
     def ptr(self) -> int:

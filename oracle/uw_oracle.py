@@ -58,8 +58,6 @@ R8  exp8 output: the true exponent byte of every element (verbatim groups
     row; nibbles of verbatim groups are 0.
 R9  GEMM: y[b, n] = sum_k W[n, k] * x[b, k] evaluated in float64 on the exact
     BF16 values.  MLP block: y = W_down (SiLU(W_gate x) * (W_up x)), float64.
-R10 Direct-palette pack: the load-time form is one record per 128 x 64 tile
-    (see direct_pack).
 """
 from __future__ import annotations
 
@@ -556,66 +554,6 @@ def rebuild_from_idx4(enc: Encoded, idx4: np.ndarray) -> np.ndarray:
     nib[:, 1::2] = idx4 >> 4
     w = rebuild_from_sm(enc.sm, enc.cb.palette[nib])
     return np.where(_verbatim_mask(enc), _verbatim_words(enc), w).astype(np.uint16)
-
-
-# ---------------------------------------------------------------------------
-# Direct-palette pack (R10): the load-time form the reconstructive GEMM
-# streams, one record per 128-row x 64-column tile
-# ---------------------------------------------------------------------------
-
-PACK_SM, PACK_IDX, PACK_MASK, PACK_VERB, PACK_VCAP = 0, 8192, 12288, 12416, 32
-
-
-def direct_pack(enc: Encoded, idx4: np.ndarray):
-    """Records of the direct-palette pack and their offsets (16-byte units).
-
-    R10 (a layout reading: the page fixes what is staged -- sign+mantissa
-    bytes, palette indices, verbatim rows -- not its byte order): tiles in
-    (row block, column block) order; per record the tile's 128x64 sm bytes
-    with the 16-byte chunk j of row r at r*64 + 16*(j ^ ((r>>1)&3)), its
-    128x32 idx4 bytes at 8192 + r*32 + 16*(j ^ ((r>>2)&1)), a 128-bit mask
-    of its verbatim rows at 12288, zeros up to 12416 (every record stays
-    128-byte aligned), then its first min(n, 32) verbatim rows.
-    Rows past the matrix are zero.
-    """
-    rows, cols = enc.rows, enc.cols
-    KB = cols // GROUP
-    MT = -(-rows // 128)
-    vg = _verbatim_mask(enc)[:, ::GROUP]                   # [rows, KB]
-    vwords = _verbatim_words(enc).reshape(rows, KB, GROUP)
-    sm = enc.sm.reshape(rows, cols)
-    recs, offs = [], [0]
-    for mt in range(MT):
-        for kb in range(KB):
-            rec_sm = np.zeros(8192, np.uint8)
-            rec_ix = np.zeros(4096, np.uint8)
-            mask = np.zeros(128, bool)
-            verb = []
-            for r in range(128):
-                n = mt * 128 + r
-                if n >= rows:
-                    continue
-                row_sm = sm[n, kb * 64:(kb + 1) * 64]
-                for j in range(4):
-                    c = r * 64 + 16 * (j ^ ((r >> 1) & 3))
-                    rec_sm[c:c + 16] = row_sm[16 * j:16 * j + 16]
-                row_ix = idx4[n, kb * 32:(kb + 1) * 32]
-                for j in range(2):
-                    c = r * 32 + 16 * (j ^ ((r >> 2) & 1))
-                    rec_ix[c:c + 16] = row_ix[16 * j:16 * j + 16]
-                if vg[n, kb]:
-                    mask[r] = True
-                    if len(verb) < PACK_VCAP:
-                        verb.append(vwords[n, kb])
-            mwords = np.zeros(4, np.uint32)
-            for r in np.flatnonzero(mask):
-                mwords[r // 32] |= np.uint32(1) << np.uint32(r % 32)
-            parts = [rec_sm, rec_ix, mwords.view(np.uint8), np.zeros(PACK_VERB - PACK_MASK - 16, np.uint8)]
-            parts += [np.ascontiguousarray(v).view(np.uint8) for v in verb]
-            rec = np.concatenate(parts)
-            recs.append(rec)
-            offs.append(offs[-1] + rec.size // 16)
-    return np.concatenate(recs), np.array(offs, dtype=np.uint32)
 
 
 # ---------------------------------------------------------------------------

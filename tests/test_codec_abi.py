@@ -12,6 +12,8 @@ from mlp_huffman_coded_b200 import synth
 from mlp_huffman_coded_b200 import uw
 from oracle import uw_oracle as O
 
+from pack_reader import verbatim_rows_per_tile
+
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
@@ -191,11 +193,15 @@ def test_oracle_decodes_the_library_stream():
 
 
 @pytest.mark.parametrize("rows,cols,rate", [(256, 512, 5e-4), (200, 640, 2e-2), (128, 64, 0.3)])
-def test_direct_pack_offsets_match_oracle(rows, cols, rate):
+def test_direct_pack_offsets_count_verbatim_rows_per_tile(rows, cols, rate):
+    """pack_off[t] = verbatim groups of all tiles before t; the pack is one
+    12304-byte body per tile plus 128 bytes per verbatim group (uw.h)."""
     w = synth.weight_matrix(rows, cols, 0.02, rate, 300.0, rows)
     enc = uw.encode(w)
     off, total = enc.pack_offsets()
-    ref = O.encode(w)
-    pack, ref_off = O.direct_pack(ref, O.transcode_palette(ref, lockstep=False))
-    assert np.array_equal(off, ref_off)
-    assert total == pack.size == 16 * int(ref_off[-1])
+    vg = O.verbatim_groups(w, O.build_palette(w))
+    ref = verbatim_rows_per_tile(vg)
+    assert np.array_equal(off, ref)
+    n_tiles = -(-rows // 128) * (cols // 64)
+    assert int(ref[-1]) == int(vg.sum()) == int(enc.layout.n_verbatim)
+    assert total == n_tiles * 12304 + 128 * int(ref[-1])

@@ -9,6 +9,7 @@ from mlp_huffman_coded_b200 import uw
 from oracle import uw_oracle as O
 
 from gpu_util import device_matrix, to_dev, to_host_u16, empty_bf16
+from pack_reader import unpack_to_w
 
 pytestmark = pytest.mark.gpu
 
@@ -129,11 +130,39 @@ def test_garbage_stream_stays_in_bounds():
     assert ws.status() == uw.UW_ERR_CORRUPT
 
 
-@pytest.mark.parametrize("rows,cols,rate", [(256, 512, 5e-4), (200, 640, 2e-2), (384, 4096, 1e-4)])
-def test_direct_pack_bit_exact(rows, cols, rate):
+@pytest.mark.parametrize("rows,cols,rate", [(256, 512, 5e-4), (200, 640, 2e-2), (384, 4096, 1e-4),
+                                           (128, 128, 0.5)])
+def test_direct_pack_reads_back_as_w(rows, cols, rate):
+    """The load-time pack, read by an independent reader of the documented
+    layout, gives back every BF16 word of W (the plain definition)."""
     w = synth.weight_matrix(rows, cols, 0.02, rate, 300.0, rows + 1)
     dm = device_matrix(w)
-    ref = O.encode(w)
-    pack, off = O.direct_pack(ref, O.transcode_palette(ref, lockstep=False))
-    assert np.array_equal(dm.pack_off.cpu().numpy().view(np.uint32), off)
-    assert np.array_equal(dm.pack.cpu().numpy(), pack)
+    off = dm.pack_off.cpu().numpy().view(np.uint32)
+    got = unpack_to_w(rows, cols, np.array(list(dm.enc.cb.palette)), dm.pack.cpu().numpy(), off)
+    assert np.array_equal(got, w)
+
+
+def test_prefixes_pointing_outside_the_store_are_reported_not_faulted():
+    """Flag prefixes tampered on the host after encoding (uploaded without
+    uw_validate) point verbatim groups past the store: the decoders and the
+    run-time transcode GEMM report UW_ERR_CORRUPT and read nothing outside
+    the store."""
+    import torch
+    w = synth.weight_matrix(256, 1024, 0.02, 3e-3, 100.0, 12)
+    enc = uw.encode(w)
+    assert enc.layout.n_verbatim > 0
+    enc.vprefix[1:] += np.uint32(1 << 24)
+    dm = uw.DeviceMatrix(enc)
+    ws = uw.Workspace(256)
+    out = empty_bf16(256 * 1024)
+    uw.decode_full(dm, out, ws)
+    assert ws.status() == uw.UW_ERR_CORRUPT
+    e8 = torch.empty(256 * 1024, dtype=torch.uint8, device="cuda")
+    uw.decode_exponent_only(dm, e8, ws)
+    assert ws.status() == uw.UW_ERR_CORRUPT
+    x = to_dev(synth.activations(4, 1024, 13))
+    y = empty_bf16(4, 256)
+    wsg = uw.Workspace(uw.workspace_bytes(dm, uw.PIPE_TRANSCODE, 4))
+    uw.gemm(dm, uw.PIPE_TRANSCODE, x, y, wsg)
+    assert wsg.status() == uw.UW_ERR_CORRUPT
+    assert wsg.status() == uw.UW_OK

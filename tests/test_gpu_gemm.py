@@ -11,7 +11,7 @@ from mlp_huffman_coded_b200 import synth
 from mlp_huffman_coded_b200 import uw
 from oracle import uw_oracle as O
 
-from gpu_util import device_matrix, empty_bf16, gemm_all, to_dev, to_host_u16, within_tol
+from gpu_util import device_matrix, empty_bf16, gemm_all, gemm_ref, to_dev, to_host_u16, within_tol
 
 pytestmark = pytest.mark.gpu
 
@@ -20,9 +20,9 @@ def _check_gemm(w, x, dm=None, pipelines=(0, 1, 2, 3)):
     if dm is None:
         dm = device_matrix(w)
     ys = gemm_all(dm, to_dev(x), pipelines)
-    y_ref = O.gemm(w, x)
+    y_ref, acc = gemm_ref(w, x)
     first = ys[pipelines[0]]
-    ok, err, rms = within_tol(first, y_ref)
+    ok, err, rms = within_tol(first, y_ref, acc)
     assert ok, (err, rms)
     for p in pipelines[1:]:
         assert np.array_equal(ys[p], first), f"pipeline {p} differs from {pipelines[0]}"
@@ -145,7 +145,7 @@ def test_full_size_mlp_matrices(which, B):
     y = empty_bf16(B, w.shape[0])
     uw.gemm_direct_palette(dm, to_dev(x), y, ws)
     ws.check()
-    ok, err, rms = within_tol(to_host_u16(y), O.gemm(w, x))
+    ok, err, rms = within_tol(to_host_u16(y), *gemm_ref(w, x))
     assert ok, (err, rms)
     if B == 8:
         ys = gemm_all(dm, to_dev(x))
@@ -187,3 +187,24 @@ def test_argument_errors():
     with pytest.raises(uw.UwError) as e:
         uw.gemm_direct_palette(dm, x, y, ws)
     assert e.value.status == uw.UW_ERR_INVALID_ARG
+
+
+def test_pack_offsets_pointing_outside_the_pack_are_reported_not_faulted():
+    """Verbatim-row offsets of the direct-palette pack tampered on the device:
+    the GEMM reports UW_ERR_CORRUPT, copies nothing outside the pack, and the
+    workspace is usable again after the status is read."""
+    w = synth.weight_matrix(512, 2048, 0.02, 3e-3, 100.0, 52)
+    dm = device_matrix(w)
+    x_host = synth.activations(8, 2048, 53)
+    x = to_dev(x_host)
+    ws = uw.Workspace(uw.workspace_bytes(dm, uw.PIPE_DIRECT, 8))
+    y = empty_bf16(8, 512)
+    good = dm.pack_off.clone()
+    dm.pack_off[3:40] = 2 ** 31 - 1
+    uw.gemm_direct_palette(dm, x, y, ws)
+    assert ws.status() == uw.UW_ERR_CORRUPT
+    dm.pack_off.copy_(good)
+    uw.gemm_direct_palette(dm, x, y, ws)
+    ws.check("after restoring the offsets")
+    ok, err, rms = within_tol(to_host_u16(y), *gemm_ref(w, x_host))
+    assert ok, (err, rms)

@@ -454,103 +454,3 @@ def test_pins_catch_planted_mistakes(mutation, check):
     m = mutated(**mutation)
     with pytest.raises(Exception):
         check(m)
-
-
-# ---------------------------------------------------------------------------
-# direct-palette pack: unpacking every record must give back W exactly
-# ---------------------------------------------------------------------------
-
-def _unpack_records_to_w(rows, cols, palette, pack, offs, orc=None):
-    """Independent reader of the documented record layout: sm chunk j of
-    row r at r*64 + 16*(j ^ ((r>>1)&3)), index chunk j at
-    8192 + r*32 + 16*(j ^ ((r>>2)&1)) (low nibble = even element), mask of
-    verbatim rows at 12288, then the first min(n, 32) verbatim rows of the
-    tile, 128 bytes each.  Returns (words, rows_in_records) where words has
-    -1 for verbatim rows beyond the 32 staged ones."""
-    KB = cols // 64
-    out = np.full((rows, cols), -1, dtype=np.int64)
-    t = 0
-    for mt in range(-(-rows // 128)):
-        for kb in range(KB):
-            rec = pack[int(offs[t]) * 16:int(offs[t + 1]) * 16]
-            t += 1
-            mask = int.from_bytes(rec[12288:12304].tobytes(), "little")
-            nv = bin(mask).count("1")
-            assert rec.size == 12416 + 128 * min(nv, 32)
-            assert not rec[12304:12416].any()
-            verb_seen = 0
-            for r in range(128):
-                n = mt * 128 + r
-                sm = np.concatenate([rec[r * 64 + 16 * (j ^ ((r >> 1) & 3)):][:16] for j in range(4)])
-                ix = np.concatenate([rec[8192 + r * 32 + 16 * (j ^ ((r >> 2) & 1)):][:16] for j in range(2)])
-                if n >= rows:
-                    assert not sm.any() and not ix.any() and not (mask >> r) & 1
-                    continue
-                if (mask >> r) & 1:
-                    if verb_seen < 32:
-                        base = 12416 + 128 * verb_seen
-                        out[n, kb * 64:(kb + 1) * 64] = rec[base:base + 128].view(np.uint16)
-                    verb_seen += 1
-                    continue
-                nib = np.empty(64, dtype=np.int64)
-                nib[0::2] = ix & 0xF
-                nib[1::2] = ix >> 4
-                e = np.asarray(palette, dtype=np.int64)[nib]
-                mant = sm.astype(np.int64) >> 1
-                sign = (sm.astype(np.int64) & 1).reshape(32, 2)[:, ::-1].reshape(64)
-                out[n, kb * 64:(kb + 1) * 64] = (sign << 15) | (e << 7) | mant
-    assert t == len(offs) - 1
-    return out
-
-
-def _verbatim_heavy(rows=128, cols=128, n_bad=40):
-    w = synth.weight_matrix(rows, cols, 0.02, 0.0, 1.0, seed=5)
-    # one distinct rare exponent (160, 161, ...; each used once, so none can
-    # enter the top-16 palette) in group 0 of each of the first n_bad rows
-    for i in range(n_bad):
-        w[i, 3] = np.uint16((160 + i) << 7)
-    return w
-
-
-def check_pack_round_trip(orc, w):
-    enc = orc.encode(w)
-    pack, offs = orc.direct_pack(enc, orc.transcode_palette(enc))
-    got = _unpack_records_to_w(w.shape[0], w.shape[1], enc.cb.palette, pack, offs)
-    staged = got >= 0
-    assert np.array_equal(got[staged], w.astype(np.int64)[staged])
-    # only verbatim rows beyond the 32 staged per tile are left to the store
-    assert not (~staged).any() or (w.shape[0] >= 33)
-    return int((~staged).sum())
-
-
-@pytest.mark.parametrize("case", ["small", "ragged", "verbatim_heavy"])
-def test_direct_pack_unpacks_to_w(case):
-    if case == "small":
-        w = synth.weight_matrix(256, 512, 0.02, 5e-4, 200.0, seed=0)
-    elif case == "ragged":
-        w = synth.weight_matrix(200, 192, 0.02, 2e-3, 100.0, seed=3)
-    else:
-        w = _verbatim_heavy()
-    left = check_pack_round_trip(O, w)
-    if case == "verbatim_heavy":
-        assert left == 8 * 64  # 40 verbatim rows in one tile: 8 beyond the 32 staged
-
-
-def _pack_mask_misplaced(enc, idx4):
-    pack, offs = O.direct_pack(enc, idx4)
-    pack = pack.copy()
-    for t in range(len(offs) - 1):
-        b = int(offs[t]) * 16
-        pack[b + 12288:b + 12304] = np.roll(pack[b + 12288:b + 12304], 1)
-    return pack, offs
-
-
-def _pack_nibbles_swapped(enc, idx4):
-    return O.direct_pack(enc, ((idx4 >> 4) | (idx4 << 4)).astype(np.uint8))
-
-
-@pytest.mark.parametrize("planted", [_pack_mask_misplaced, _pack_nibbles_swapped])
-def test_pack_pin_catches_planted_mistakes(planted):
-    m = mutated(direct_pack=planted)
-    with pytest.raises(AssertionError):
-        check_pack_round_trip(m, synth.weight_matrix(256, 512, 0.02, 5e-4, 200.0, seed=0))
