@@ -56,7 +56,7 @@ namespace {
 // `groups` rebuild warpgroups of 4 warps (group g rebuilds stages i with
 // i % groups == g, so several stages are rebuilt at once), then 4 epilogue
 // warps.
-constexpr int kMaxGroups = 2;
+constexpr int kMaxGroups = 3;
 constexpr int kMaxThreads = 32 * (6 + 4 * kMaxGroups);
 constexpr int kWarpProducer = 0;
 constexpr int kWarpMma = 1;
@@ -193,7 +193,18 @@ __device__ __forceinline__ bool group_and(bool v) {  // the 4 epilogue warps (na
 }
 __device__ __forceinline__ void group_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
-__device__ __forceinline__ uint4 lds128(const uint8_t* p) { return *reinterpret_cast<const uint4*>(p); }
+// Shared-memory loads at 32-bit shared-window addresses (ld.shared, never a
+// generic load; volatile keeps them after the barrier waits that order them).
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
 
 // y[b, n] = bf16(v), or bf16(SiLU(gate[b, n]) * bf16(v)) for the fused
 // SwiGLU epilogue.
@@ -218,8 +229,8 @@ __device__ __forceinline__ int mask_below(const uint4& m, int q) {
 // 2i in the low half of word i), ready for tcgen05.st.  Tile rows arrive with
 // a swizzle that keeps these row-per-thread 16-byte reads bank-conflict free.
 
-__device__ __forceinline__ void rebuild_idx_row(const PaletteTables& pal, bool uniform, const uint8_t* ts,
-                                                const uint8_t* ti, int r, uint32_t (&o)[32]) {
+__device__ __forceinline__ void rebuild_idx_row(const PaletteTables& pal, bool uniform, uint32_t ts, uint32_t ti,
+                                                int r, uint32_t (&o)[32]) {
   uint32_t iw[8];
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
@@ -251,10 +262,9 @@ __device__ __forceinline__ void rebuild_idx_row(const PaletteTables& pal, bool u
 }
 
 template <int L>
-__device__ __forceinline__ void rebuild_row(const uint8_t* stage, const KParams& p, int r, int j,
-                                            uint32_t (&o)[32]) {
+__device__ __forceinline__ void rebuild_row(uint32_t stage, const KParams& p, int r, int j, uint32_t (&o)[32]) {
   if constexpr (L == kBF16) {
-    const uint8_t* t = stage + p.off_wa + j * 16384;  // rows of 128 B, 128-byte swizzle
+    const uint32_t t = stage + p.off_wa + j * 16384;  // rows of 128 B, 128-byte swizzle
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       const uint4 v = lds128(t + r * 128 + ((c ^ (r & 7)) << 4));
@@ -264,8 +274,8 @@ __device__ __forceinline__ void rebuild_row(const uint8_t* stage, const KParams&
       o[4 * c + 3] = v.w;
     }
   } else if constexpr (L == kEXP8) {
-    const uint8_t* ts = stage + p.off_wa + j * 8192;  // sm rows of 64 B, 64-byte swizzle
-    const uint8_t* te = stage + p.off_wb + j * 8192;  // exponent rows of 64 B, 64-byte swizzle
+    const uint32_t ts = stage + p.off_wa + j * 8192;  // sm rows of 64 B, 64-byte swizzle
+    const uint32_t te = stage + p.off_wb + j * 8192;  // exponent rows of 64 B, 64-byte swizzle
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
       const int off = (c ^ ((r >> 1) & 3)) << 4;
@@ -277,7 +287,7 @@ __device__ __forceinline__ void rebuild_row(const uint8_t* stage, const KParams&
       rebuild4(s.w, e.w, o[8 * c + 6], o[8 * c + 7]);
     }
   } else if constexpr (loader_pack(L)) {
-    const uint8_t* body = stage + p.off_wa + j * kBody;
+    const uint32_t body = stage + p.off_wa + j * kBody;
     rebuild_idx_row(p.pal, loader_uniform(L), body, body + kBodyIdx, r, o);
   } else {
     // run-time transcode: sm rows of 64 B (64-byte swizzle), index rows of
@@ -286,10 +296,20 @@ __device__ __forceinline__ void rebuild_row(const uint8_t* stage, const KParams&
   }
 }
 
-__device__ __forceinline__ void copy_row(const uint4* src, uint32_t (&o)[32]) {
+__device__ __forceinline__ void copy_row(const uint4* src, uint32_t (&o)[32]) {  // global
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     const uint4 v = src[c];
+    o[4 * c] = v.x;
+    o[4 * c + 1] = v.y;
+    o[4 * c + 2] = v.z;
+    o[4 * c + 3] = v.w;
+  }
+}
+__device__ __forceinline__ void copy_row_s(uint32_t src, uint32_t (&o)[32]) {  // shared
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint4 v = lds128(src + 16 * c);
     o[4 * c] = v.x;
     o[4 * c + 1] = v.y;
     o[4 * c + 2] = v.z;
@@ -305,8 +325,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
                 const __grid_constant__ CUtensorMap tm_g, const KParams p) {
   constexpr bool kIdx4 = loader_idx4(L);  // row-major indices + verbatim store
   constexpr bool kPack = loader_pack(L);
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 1024-byte aligned base (the 128-byte swizzle repeats every 1024 bytes),
+  // derived from the shared array so accesses stay in the shared space
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  const uint32_t smem_s = smem_u32(smem);
   Bars* bars = reinterpret_cast<Bars*>(smem + p.bar_off);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -360,12 +383,26 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     }
   };
 
-  // ---- set-up.  The producer thread initialises the barriers and at once
-  // issues the weight copies of the first stages (their phases cannot
-  // complete before its own arrive, which follows once the tables are in);
-  // the MMA warp allocates tensor memory meanwhile.
+  // ---- set-up.  The producer warp first sends the loads of this CTA's
+  // pack_off entries (they must not queue behind the weight stream), then its
+  // first thread initialises the barriers and issues the weight copies of
+  // the first kEarlyStages stages (their phases cannot complete before its
+  // own arrive, which follows once the table is in); the MMA warp allocates
+  // tensor memory meanwhile.  Only a few stages go out before the main loop:
+  // copies issued together land in no useful order, so a large first burst
+  // delays the first stage.
+  constexpr int kEarlyStages = 2;
   int early = 0;  // stages whose weights are already in flight
   if (warp == kWarpProducer) {
+    const int64_t n_tiles_total = static_cast<int64_t>((p.N + 127) / 128) * p.KB;
+    const int64_t want = static_cast<int64_t>(mt_last - mt_first + 1) * p.KB + 1;
+    const int64_t cnt = kPack ? (want < p.n_soff ? want : p.n_soff) : 0;
+    uint32_t v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int64_t w = j * 32 + lane;
+      v[j] = (w < cnt && pt_min + w <= n_tiles_total) ? __ldg(p.pack_off + pt_min + w) : 0u;
+    }
     if (lane == 0) {
       for (int s = 0; s < S; ++s) {
         mbar_init(&bars->full[s], 1);
@@ -388,7 +425,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       if constexpr (!kIdx4) {
         StageWalk w;
         walk_init(w, u0, u1, p);
-        for (; early < S && w.u < u1; ++early, walk_next(w, u1, p)) {
+        for (; early < kEarlyStages && early < S && w.u < u1; ++early, walk_next(w, u1, p)) {
           mbar_expect_tx(&bars->full[early], weight_bytes(w));
           issue_weights(early, w);
         }
@@ -400,13 +437,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       if (L != kBF16 && !kPack) prefetch_tensormap(&tm_wb);
     }
     early = __shfl_sync(0xFFFFFFFFu, early, 0);
-    // pack: this CTA's pack_off entries (verbatim-row offsets of its tiles)
     if (kPack) {
-      const int64_t n_tiles_total = static_cast<int64_t>((p.N + 127) / 128) * p.KB;
-      const int64_t want = static_cast<int64_t>(mt_last - mt_first + 1) * p.KB + 1;
-      const int64_t cnt = want < p.n_soff ? want : p.n_soff;
-      for (int64_t w0 = 0; w0 < cnt; w0 += 256) {
-        uint32_t v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int64_t w = j * 32 + lane;
+        if (w < cnt) soff[w] = v[j];
+      }
+      // a CTA spanning more than two row tiles of a short matrix: the rest
+      for (int64_t w0 = 256; w0 < cnt; w0 += 256) {
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int64_t w = w0 + j * 32 + lane;
@@ -706,7 +744,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       if (turn != grp) continue;
       if (!warp_wait(&bars->full[s], k & 1, bars, p.status)) break;
       tc_fence_after();
-      const uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
+      const uint32_t stage = smem_s + static_cast<uint32_t>(s) * p.stage_bytes;
       int vbase = 0;  // pack: verbatim rows of the stage's earlier k-blocks
 #pragma unroll 1
       for (int j = 0; j < w.n; ++j) {
@@ -719,11 +757,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           if ((m >> lane) & 1) {
             const int idx = vbase + mask_below(mk, q) + __popc(m & ((1u << lane) - 1));
             if (idx < p.vcap) {
-              copy_row(reinterpret_cast<const uint4*>(stage + p.off_verb + idx * 128), o);
+              copy_row_s(stage + p.off_verb + idx * 128, o);
             } else {
               // more verbatim rows than staged ones: this one from HBM
               const int64_t slot = static_cast<int64_t>(w.mt) * p.KB + w.kb - pt_min;
-              const long long g = static_cast<long long>(soff[slot]) + idx;
+              const long long g = static_cast<long long>(lds32(smem_s + p.soff_off + 4u * static_cast<uint32_t>(slot))) + idx;
               if (g < p.n_verbatim)
                 copy_row(reinterpret_cast<const uint4*>(p.tails + static_cast<uint64_t>(g) * 128u), o);
               else
@@ -732,13 +770,12 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           }
           vbase += __popc(mk.x) + __popc(mk.y) + __popc(mk.z) + __popc(mk.w);
         } else if constexpr (kIdx4) {
-          const uint32_t* hdr = reinterpret_cast<const uint32_t*>(stage + p.off_hdr);
-          const uint32_t m = hdr[q];
+          const uint4 hdr = lds128(stage + p.off_hdr);
+          const uint32_t m = mask_word(hdr, q);
           if ((m >> lane) & 1) {
-            int idx = __popc(m & ((1u << lane) - 1));
-            for (int qq = 0; qq < q; ++qq) idx += __popc(hdr[qq]);
+            const int idx = mask_below(hdr, q) + __popc(m & ((1u << lane) - 1));
             if (idx < p.vcap) {
-              copy_row(reinterpret_cast<const uint4*>(stage + p.off_verb + idx * 128), o);
+              copy_row_s(stage + p.off_verb + idx * 128, o);
             } else {
               // more verbatim rows than staged slots: read this one from HBM
               const int64_t n = static_cast<int64_t>(w.mt) * 128 + r;
@@ -954,7 +991,7 @@ __global__ void swiglu_kernel(const __nv_bfloat16* __restrict__ g, const __nv_bf
 // ------------------------------ host side ------------------------------------
 
 struct Layout {
-  int stages = 0, ks = 1;
+  int stages = 0, ks = 1, groups = 1;
   uint32_t stage_bytes = 0, off_x = 0, off_wa = 0, off_wb = 0, off_verb = 0, off_hdr = 0;
   uint32_t x_kb_bytes = 0;
   uint32_t meta_off = 0, meta_slot_words = 0, bar_off = 0, soff_off = 0, a_col0 = 0, epi_off = 0;
@@ -1046,6 +1083,12 @@ bool make_layout(int loader, const GemmPlan& plan, int wpr, bool tma_out, bool g
   int stages = static_cast<int>((kSmemLimit - fixed) / l.stage_bytes);
   stages = std::min({stages, max_stages(), tmem_stages});
   if (stages < 2) return false;
+  // Rebuild group g takes the stages i with i % groups == g.  A group may
+  // only wait for a ring slot's next phase once its current phase has
+  // completed (the wait tests a phase parity), which holds when every slot
+  // always belongs to the same group: stages must be a multiple of groups.
+  l.groups = std::min(rebuild_groups(), stages);
+  stages -= stages % l.groups;
   l.stages = stages;
   if (pack) {
     // spread the remaining shared memory over the stages as on-chip verbatim
@@ -1238,7 +1281,7 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.partials = reinterpret_cast<float*>(ws + kWsHeader + plan.counter_bytes);
   kp.pal = pal;
   kp.idesc = idesc_bf16_f32(plan.ntile);
-  kp.groups = rebuild_groups();
+  kp.groups = lay.groups;
   kp.vcap = lay.vcap;
   kp.n_acc = 2 * plan.ntile <= 256 ? 2 : 1;
   kp.pack = a.pack;
