@@ -187,6 +187,17 @@ __device__ __forceinline__ bool wait_count_at_least(const uint32_t* counter, uin
   return true;
 }
 
+// Ticket: every write this thread has observed (including other threads'
+// writes ordered before it by a CTA barrier) becomes visible before the add,
+// and every write published before the adds that precede it becomes visible
+// to this thread (and, through a later CTA barrier, to the others).  Returns
+// the previous value.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("fence.acq_rel.gpu;\n\tatom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
+
 // Publish: every write this thread has observed (including other threads'
 // writes ordered before it by a CTA barrier) becomes visible before the add.
 __device__ __forceinline__ void red_release_gpu_add(uint32_t* p, uint32_t v) {

@@ -52,17 +52,22 @@ namespace uw {
 
 namespace {
 
-// Warp roles: 0 = TMA producer, 1 = MMA issuer (and TMEM owner), then
-// `groups` rebuild warpgroups of 4 warps (group g rebuilds stages i with
-// i % groups == g, so several stages are rebuilt at once), then 4 epilogue
-// warps.
-constexpr int kMaxGroups = 3;
-constexpr int kMaxThreads = 32 * (6 + 4 * kMaxGroups);
+// Warp roles: 0 = weight producer, 1..4 = MMA issuers 0..3 (warp 1 owns
+// tensor memory), 5 = activation producer, then `groups` rebuild warpgroups
+// of 4 warps (group g rebuilds stages i with i % groups == g, so several
+// stages are rebuilt at once), then 4 epilogue warps.  One thread issues a
+// tcgen05.mma (M = 128, K = 16) only every ~120 cycles whatever N up to 128,
+// while several issuing threads overlap: at small batch the MMAs are spread
+// over up to 4 issuers.
+constexpr int kMaxGroups = 2;
+constexpr int kMaxIssuers = 4;
+constexpr int kMaxThreads = 32 * (10 + 4 * kMaxGroups);
 constexpr int kWarpProducer = 0;
 constexpr int kWarpMma = 1;
-constexpr int kWarpRebuild0 = 2;
+constexpr int kWarpXProducer = 5;
+constexpr int kWarpRebuild0 = 6;
 constexpr int kVCap = 16;  // run-time transcode: verbatim rows staged per k-block
-constexpr int kMaxStages = 16;
+constexpr int kMaxSlots = 16;
 constexpr int kMaxKS = 4;  // k-blocks per stage
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCol = 0;  // accumulators first; rebuilt A tiles after them
@@ -86,9 +91,12 @@ struct KParams {
   int N, K, B, KB, n_ntiles, ntile;
   long long units;
   int grid;
-  int stages;
-  int ks;  // k-blocks per stage
-  uint32_t stage_bytes, off_x, off_wa, off_wb, off_verb, off_hdr;
+  int ks;      // k-blocks per stage
+  int sw;      // weight ring slots (shared memory)
+  int sa;      // activation + A-tile ring slots (shared memory + tensor memory)
+  int n_iss;   // MMA issuers: issuer i takes the k-blocks kb with kb % n_iss == i
+  uint32_t w_slot_bytes, x_slot_bytes, w_base, x_base;
+  uint32_t off_wb, off_verb, off_hdr;  // inside a weight slot (region a at 0)
   uint32_t x_kb_bytes;  // activation tile of one k-block: ntile rows x 128 bytes
   uint32_t meta_off, meta_slot_words;  // run-time transcode: per slot flags then prefixes
   uint32_t bar_off;
@@ -119,16 +127,17 @@ struct KParams {
 };
 
 struct Bars {
-  uint64_t full[kMaxStages];
-  uint64_t rebuilt[kMaxStages];
-  uint64_t empty[kMaxStages];
-  uint64_t acc_full[2], acc_empty[2], drain;
+  uint64_t wfull[kMaxSlots];   // weight slot landed
+  uint64_t wempty[kMaxSlots];  // weight slot read by its rebuild group
+  uint64_t xfull[kMaxSlots];   // activation slot landed
+  uint64_t afull[kMaxSlots];   // A tiles of the slot rebuilt into tensor memory
+  uint64_t aempty[kMaxSlots];  // the slot's MMAs have completed (activations and A free)
+  uint64_t acc_full[2], acc_empty[2], drain[kMaxIssuers];
   uint64_t meta_full[2];
   uint64_t gate_full[2];  // fused SwiGLU: gate chunk landed
   uint32_t tmem_base;
   uint32_t abort;
-  uint32_t is_last;
-  uint32_t dep_ready;  // the previous kernel on the stream has completed
+  uint32_t last_arriver;  // epilogue: this CTA completed a split tile
 };
 
 __device__ __forceinline__ int64_t unit_begin(int64_t c, const KParams& p) {
@@ -172,6 +181,18 @@ __device__ __forceinline__ void walk_next(StageWalk& w, int64_t u1, const KParam
     }
   }
   walk_fix_n(w, u1, p);
+}
+// ring position of stage st in a ring of `slots`: slot and use count, kept
+// incrementally
+struct Ring {
+  int slot;
+  uint32_t use;
+};
+__device__ __forceinline__ void ring_next(Ring& r, int slots) {
+  if (++r.slot == slots) {
+    r.slot = 0;
+    ++r.use;
+  }
 }
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, Bars* b, uint32_t* status) {
@@ -264,7 +285,7 @@ __device__ __forceinline__ void rebuild_idx_row(const PaletteTables& pal, bool u
 template <int L>
 __device__ __forceinline__ void rebuild_row(uint32_t stage, const KParams& p, int r, int j, uint32_t (&o)[32]) {
   if constexpr (L == kBF16) {
-    const uint32_t t = stage + p.off_wa + j * 16384;  // rows of 128 B, 128-byte swizzle
+    const uint32_t t = stage + j * 16384;  // rows of 128 B, 128-byte swizzle
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       const uint4 v = lds128(t + r * 128 + ((c ^ (r & 7)) << 4));
@@ -274,7 +295,7 @@ __device__ __forceinline__ void rebuild_row(uint32_t stage, const KParams& p, in
       o[4 * c + 3] = v.w;
     }
   } else if constexpr (L == kEXP8) {
-    const uint32_t ts = stage + p.off_wa + j * 8192;  // sm rows of 64 B, 64-byte swizzle
+    const uint32_t ts = stage + j * 8192;  // sm rows of 64 B, 64-byte swizzle
     const uint32_t te = stage + p.off_wb + j * 8192;  // exponent rows of 64 B, 64-byte swizzle
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
@@ -287,12 +308,12 @@ __device__ __forceinline__ void rebuild_row(uint32_t stage, const KParams& p, in
       rebuild4(s.w, e.w, o[8 * c + 6], o[8 * c + 7]);
     }
   } else if constexpr (loader_pack(L)) {
-    const uint32_t body = stage + p.off_wa + j * kBody;
+    const uint32_t body = stage + j * kBody;
     rebuild_idx_row(p.pal, loader_uniform(L), body, body + kBodyIdx, r, o);
   } else {
     // run-time transcode: sm rows of 64 B (64-byte swizzle), index rows of
     // 32 B (32-byte swizzle)
-    rebuild_idx_row(p.pal, loader_uniform(L), stage + p.off_wa + j * 8192, stage + p.off_wb + j * 4096, r, o);
+    rebuild_idx_row(p.pal, loader_uniform(L), stage + j * 8192, stage + p.off_wb + j * 4096, r, o);
   }
 }
 
@@ -335,7 +356,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   const int lane = threadIdx.x & 31;
   const int64_t u0 = unit_begin(blockIdx.x, p);
   const int64_t u1 = unit_begin(blockIdx.x + 1, p);
-  const int S = p.stages;
+  const int SW = p.sw, SA = p.sa;
   const int G = p.groups;
   const int warp_epi0 = kWarpRebuild0 + 4 * G;
 
@@ -343,6 +364,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   const int mt_last = static_cast<int>(((u1 - 1) / p.KB) / p.n_ntiles);
   uint32_t* soff = reinterpret_cast<uint32_t*>(smem + p.soff_off);
   const int64_t pt_min = static_cast<int64_t>(mt_first) * p.KB;
+  auto wslot = [&](int s) -> uint8_t* { return smem + p.w_base + static_cast<size_t>(s) * p.w_slot_bytes; };
 
   // Weight bytes of a stage, and their copies (every loader but the run-time
   // transcode, whose verbatim rows need the flag tables first).
@@ -353,44 +375,36 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   };
   const uint64_t stream_policy = l2_evict_first();
   auto issue_weights = [&](int s, const StageWalk& w) {
-    uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
+    uint8_t* slot = wslot(s);
+    uint64_t* bar = &bars->wfull[s];
     if constexpr (kPack) {
       const int64_t tile = static_cast<int64_t>(w.mt) * p.KB + w.kb;
-      bulk_load_hint(stage + p.off_wa, p.pack + static_cast<uint64_t>(tile) * kBody, static_cast<uint32_t>(w.n) * kBody,
-                     &bars->full[s], stream_policy);
+      bulk_load_hint(slot, p.pack + static_cast<uint64_t>(tile) * kBody, static_cast<uint32_t>(w.n) * kBody, bar,
+                     stream_policy);
     } else {
       for (int j = 0; j < w.n; ++j) {
         const int c = (w.kb + j) * 64;
         if constexpr (L == kBF16) {
-          tma_load_2d(stage + p.off_wa + j * 16384, &tm_wa, c, w.mt * 128, &bars->full[s]);
+          tma_load_2d(slot + j * 16384, &tm_wa, c, w.mt * 128, bar);
         } else if constexpr (L == kEXP8) {
-          tma_load_2d(stage + p.off_wa + j * 8192, &tm_wa, c, w.mt * 128, &bars->full[s]);
-          tma_load_2d(stage + p.off_wb + j * 8192, &tm_wb, c, w.mt * 128, &bars->full[s]);
+          tma_load_2d(slot + j * 8192, &tm_wa, c, w.mt * 128, bar);
+          tma_load_2d(slot + p.off_wb + j * 8192, &tm_wb, c, w.mt * 128, bar);
         } else {
-          tma_load_2d(stage + p.off_wa + j * 8192, &tm_wa, c, w.mt * 128, &bars->full[s]);
-          tma_load_2d(stage + p.off_wb + j * 4096, &tm_wb, c / 2, w.mt * 128, &bars->full[s]);
+          tma_load_2d(slot + j * 8192, &tm_wa, c, w.mt * 128, bar);
+          tma_load_2d(slot + p.off_wb + j * 4096, &tm_wb, c / 2, w.mt * 128, bar);
         }
       }
     }
   };
-  auto issue_x = [&](int s, const StageWalk& w) {
-    uint8_t* dst = smem + static_cast<size_t>(s) * p.stage_bytes + p.off_x;
-    if (p.x3d) {
-      tma_load_3d(dst, &tm_x, 0, w.nt * p.ntile, w.kb, &bars->full[s]);
-    } else {
-      for (int j = 0; j < p.ks; ++j)
-        tma_load_2d(dst + j * p.x_kb_bytes, &tm_x, (w.kb + j) * 64, w.nt * p.ntile, &bars->full[s]);
-    }
-  };
 
-  // ---- set-up.  The producer warp first sends the loads of this CTA's
-  // pack_off entries (they must not queue behind the weight stream), then its
-  // first thread initialises the barriers and issues the weight copies of
-  // the first kEarlyStages stages (their phases cannot complete before its
-  // own arrive, which follows once the table is in); the MMA warp allocates
-  // tensor memory meanwhile.  Only a few stages go out before the main loop:
-  // copies issued together land in no useful order, so a large first burst
-  // delays the first stage.
+  // ---- set-up.  The weight producer warp first sends the loads of this
+  // CTA's pack_off entries (they must not queue behind the weight stream),
+  // then its first thread initialises the barriers and issues the weight
+  // copies of the first kEarlyStages stages (their phases cannot complete
+  // before its own arrive, which follows once the table is in); the MMA warp
+  // allocates tensor memory meanwhile.  Only a few stages go out before the
+  // main loop: copies issued together land in no useful order, so a large
+  // first burst delays the first stage.
   constexpr int kEarlyStages = 2;
   int early = 0;  // stages whose weights are already in flight
   if (warp == kWarpProducer) {
@@ -404,35 +418,32 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       v[j] = (w < cnt && pt_min + w <= n_tiles_total) ? __ldg(p.pack_off + pt_min + w) : 0u;
     }
     if (lane == 0) {
-      for (int s = 0; s < S; ++s) {
-        mbar_init(&bars->full[s], 1);
-        mbar_init(&bars->rebuilt[s], 4);
-        mbar_init(&bars->empty[s], 1);
+      for (int s = 0; s < SW; ++s) {
+        mbar_init(&bars->wfull[s], 1);
+        mbar_init(&bars->wempty[s], 4);
       }
-      mbar_init(&bars->acc_full[0], 1);
-      mbar_init(&bars->acc_full[1], 1);
-      mbar_init(&bars->acc_empty[0], 4);
-      mbar_init(&bars->acc_empty[1], 4);
-      mbar_init(&bars->drain, 1);
-      mbar_init(&bars->meta_full[0], 1);
-      mbar_init(&bars->meta_full[1], 1);
-      mbar_init(&bars->gate_full[0], 1);
-      mbar_init(&bars->gate_full[1], 1);
+      for (int s = 0; s < SA; ++s) {
+        mbar_init(&bars->xfull[s], 1);
+        mbar_init(&bars->afull[s], 4);
+        mbar_init(&bars->aempty[s], p.n_iss);
+      }
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&bars->acc_full[i], p.n_iss);
+        mbar_init(&bars->acc_empty[i], 4);
+        mbar_init(&bars->meta_full[i], 1);
+        mbar_init(&bars->gate_full[i], 1);
+      }
+      for (int i = 0; i < kMaxIssuers; ++i) mbar_init(&bars->drain[i], 1);
       bars->abort = 0;
-      bars->is_last = 0;
-      bars->dep_ready = 0;
       mbar_fence_init();
       if constexpr (!kIdx4) {
         StageWalk w;
         walk_init(w, u0, u1, p);
-        for (; early < kEarlyStages && early < S && w.u < u1; ++early, walk_next(w, u1, p)) {
-          mbar_expect_tx(&bars->full[early], weight_bytes(w));
+        for (; early < kEarlyStages && early < SW && w.u < u1; ++early, walk_next(w, u1, p)) {
+          mbar_expect_tx(&bars->wfull[early], weight_bytes(w));
           issue_weights(early, w);
         }
       }
-      prefetch_tensormap(&tm_x);
-      if (p.tma_out) prefetch_tensormap(&tm_y);
-      if (p.tma_out && p.gate) prefetch_tensormap(&tm_g);
       if (!kPack) prefetch_tensormap(&tm_wa);
       if (L != kBF16 && !kPack) prefetch_tensormap(&tm_wb);
     }
@@ -458,6 +469,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       }
     }
     __syncwarp();
+  } else if (warp == kWarpXProducer && lane == 0) {
+    prefetch_tensormap(&tm_x);
+    if (p.tma_out) prefetch_tensormap(&tm_y);
+    if (p.tma_out && p.gate) prefetch_tensormap(&tm_g);
   }
   if (warp == kWarpMma) {
     tmem_alloc(&bars->tmem_base, kTmemCols);
@@ -469,47 +484,26 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == kWarpProducer) {
-    // ------------------------------ producer --------------------------------
-    // Activations may be the output of the previous kernel on the stream
-    // (programmatic dependent launch lets this kernel start while that one
-    // finishes).  Weight copies go out at once; activation tiles, which
-    // complete the same barriers, follow as soon as an epilogue thread has
-    // seen that kernel complete (dep_ready), at the latest after the S-th
-    // stage.
+    // --------------------------- weight producer ----------------------------
+    // Weights are constant: they stream from the start, independent of the
+    // kernel ahead on the stream.  A weight slot is free again once its
+    // rebuild group has read it.
     if constexpr (!kIdx4) {
       if (lane == 0) {
-        bool dep_done = false;
-        StageWalk w, wx;
+        StageWalk w;
         walk_init(w, u0, u1, p);
-        wx = w;
-        int sx = 0;          // ring slot of the first stage without its activation tile
-        int64_t x_next = 0;  // that stage's index
-        int s = 0;
-        uint32_t k = 0;
+        Ring rw{0, 0};
         int64_t st = 0;
-        auto issue_deferred_x = [&](int64_t upto) {
-          for (; x_next < upto; ++x_next) {
-            issue_x(sx, wx);
-            walk_next(wx, u1, p);
-            if (++sx == S) sx = 0;
-          }
-        };
-        for (; w.u < u1; walk_next(w, u1, p), ++st) {
-          if (st > 0 && ++s == S) {
-            s = 0;
-            ++k;
-          }
-          if (k > 0 && !mbar_wait(&bars->empty[s], (k - 1) & 1, &bars->abort, p.status)) break;
-          uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
-          uint32_t tx = static_cast<uint32_t>(p.ks) * p.x_kb_bytes;
-          const bool w_early = st < early;
-          if (!w_early) tx += weight_bytes(w);
+        for (; w.u < u1; walk_next(w, u1, p), ++st, ring_next(rw, SW)) {
+          if (rw.use > 0 && !mbar_wait(&bars->wempty[rw.slot], (rw.use - 1) & 1, &bars->abort, p.status)) break;
+          uint8_t* slot = wslot(rw.slot);
+          uint32_t tx = st < early ? 0u : weight_bytes(w);
           uint32_t t_first = 0, t_rows = 0;
           if constexpr (kPack) {
             // verbatim rows of the stage's tiles: one contiguous run
-            const int64_t slot = static_cast<int64_t>(w.mt) * p.KB + w.kb - pt_min;
-            if (slot >= 0 && slot + w.n < p.n_soff) {
-              const uint32_t a = soff[slot], b = soff[slot + w.n];
+            const int64_t sl = static_cast<int64_t>(w.mt) * p.KB + w.kb - pt_min;
+            if (sl >= 0 && sl + w.n < p.n_soff) {
+              const uint32_t a = soff[sl], b = soff[sl + w.n];
               if (b < a || b - a > 128u * static_cast<uint32_t>(w.n) || static_cast<long long>(b) > p.n_verbatim) {
                 record_status(p.status, UW_ERR_CORRUPT);
               } else {
@@ -521,32 +515,19 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             }
             tx += t_rows * 128u;
           }
-          mbar_arrive_expect_tx(&bars->full[s], tx);
-          if (!w_early) issue_weights(s, w);
+          mbar_arrive_expect_tx(&bars->wfull[rw.slot], tx);
+          if (st >= early) issue_weights(rw.slot, w);
           if (kPack && t_rows)
-            bulk_load_hint(stage + p.off_verb, p.tails + static_cast<uint64_t>(t_first) * 128u, t_rows * 128u,
-                           &bars->full[s], stream_policy);
-          if (dep_done) {
-            issue_x(s, w);
-          } else if (ld_acquire_cta(&bars->dep_ready) || st == S - 1 || w.u + w.n >= u1) {
-            griddep_wait();  // immediate once dep_ready is set; formal ordering
-            dep_done = true;
-            issue_deferred_x(st + 1);
-          }
+            bulk_load_hint(slot + p.off_verb, p.tails + static_cast<uint64_t>(t_first) * 128u, t_rows * 128u,
+                           &bars->wfull[rw.slot], stream_policy);
         }
         // stopped early (an abort): stages whose weights went out before the
-        // tables arrived still need their arrive; the previous kernel must be
-        // waited for and the issued stages' activation tiles completed
-        if (!dep_done) {
-          griddep_wait();
-          issue_deferred_x(st);
-        }
-        for (int64_t e = st; e < early; ++e) mbar_arrive(&bars->full[e]);
-        // drain: the last use of every stage must land before the CTA exits
-        // (normally already complete)
+        // table arrived still need their arrive; then every issued copy must
+        // land before the CTA exits (normally already complete)
+        for (int64_t e = st; e < early; ++e) mbar_arrive(&bars->wfull[e]);
         const int64_t issued = st > early ? st : early;
-        for (int64_t q = issued - S > 0 ? issued - S : 0; q < issued; ++q)
-          mbar_wait(&bars->full[q % S], static_cast<uint32_t>(q / S) & 1, nullptr, p.status);
+        for (int64_t q = issued - SW > 0 ? issued - SW : 0; q < issued; ++q)
+          mbar_wait(&bars->wfull[q % SW], static_cast<uint32_t>(q / SW) & 1, nullptr, p.status);
       }
       __syncwarp();
     } else {
@@ -581,33 +562,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       issue_meta(mt_first, 0);
       if (mt_first + 1 <= mt_last) issue_meta(mt_first + 1, 1);
       int cur_mt = -1;
-      bool dep_done = false;
-      StageWalk w, wx;
+      StageWalk w;
       walk_init(w, u0, u1, p);
-      wx = w;
-      int sx = 0;
-      int64_t x_next = 0;
-      int s = 0;
-      uint32_t k = 0;
+      Ring rw{0, 0};
       int64_t st = 0;
-      auto finish_dependency = [&](int64_t upto) {
-        griddep_wait();
-        dep_done = true;
-        for (; x_next < upto; ++x_next) {
-          if (lane == 0) issue_x(sx, wx);
-          walk_next(wx, u1, p);
-          if (++sx == S) sx = 0;
-        }
-        __syncwarp();
-      };
-      for (; w.u < u1; walk_next(w, u1, p), ++st) {
-        if (st > 0 && ++s == S) {
-          s = 0;
-          ++k;
-        }
-        if (k > 0 && !warp_wait(&bars->empty[s], (k - 1) & 1, bars, p.status)) break;
-        uint8_t* stage = smem + static_cast<size_t>(s) * p.stage_bytes;
-        uint32_t tx = static_cast<uint32_t>(p.ks) * p.x_kb_bytes + weight_bytes(w);
+      for (; w.u < u1; walk_next(w, u1, p), ++st, ring_next(rw, SW)) {
+        if (rw.use > 0 && !warp_wait(&bars->wempty[rw.slot], (rw.use - 1) & 1, bars, p.status)) break;
+        uint8_t* slot = wslot(rw.slot);
+        uint32_t tx = weight_bytes(w);
         const int jm = w.mt - mt_first;
         if (w.mt != cur_mt) {
           if (jm >= 1 && w.mt + 1 <= mt_last) issue_meta(w.mt + 1, (jm + 1) & 1);
@@ -618,7 +580,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         const uint32_t* mp = mf + p.meta_slot_words;
         const int fwi = w.kb >> 5;
         const uint32_t fbit = 1u << (w.kb & 31);
-        uint32_t* hdr = reinterpret_cast<uint32_t*>(stage + p.off_hdr);
+        uint32_t* hdr = reinterpret_cast<uint32_t*>(slot + p.off_hdr);
         int total = 0, n_copy = 0;
         int vq_dst[4];
         int64_t vq_src[4];
@@ -642,84 +604,113 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         tx += static_cast<uint32_t>(n_copy) * 128u;
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive_expect_tx(&bars->full[s], tx);
-          issue_weights(s, w);
-          if (dep_done) issue_x(s, w);
+          mbar_arrive_expect_tx(&bars->wfull[rw.slot], tx);
+          issue_weights(rw.slot, w);
         }
         __syncwarp();
 #pragma unroll
         for (int q = 0; q < 4; ++q)
           if (vq_dst[q] >= 0)
-            bulk_load(stage + p.off_verb + vq_dst[q] * 128, p.verbatim + vq_src[q] * 64, 128, &bars->full[s]);
-        if (!dep_done) {
-          const uint32_t ready = __shfl_sync(0xFFFFFFFFu, lane == 0 ? ld_acquire_cta(&bars->dep_ready) : 0u, 0);
-          if (ready || st == S - 1 || w.u + w.n >= u1) finish_dependency(st + 1);
-        }
+            bulk_load(slot + p.off_verb + vq_dst[q] * 128, p.verbatim + vq_src[q] * 64, 128, &bars->wfull[rw.slot]);
       }
-      if (!dep_done) finish_dependency(st);
       if (lane == 0) {
-        for (int64_t q = st - S > 0 ? st - S : 0; q < st; ++q)
-          mbar_wait(&bars->full[q % S], static_cast<uint32_t>(q / S) & 1, nullptr, p.status);
+        for (int64_t q = st - SW > 0 ? st - SW : 0; q < st; ++q)
+          mbar_wait(&bars->wfull[q % SW], static_cast<uint32_t>(q / SW) & 1, nullptr, p.status);
         for (int sl = 0; sl < 2; ++sl)
           if (meta_issued[sl] > 0) mbar_wait(&bars->meta_full[sl], (meta_issued[sl] - 1) & 1, nullptr, p.status);
       }
       __syncwarp();
     }
-  } else if (warp == kWarpMma) {
-    // ----------------------------- MMA issuer -------------------------------
-    // One thread issues every MMA: per stage it waits for the stage's copies
-    // and its rebuilt A tiles, issues 4 MMAs (K = 16 each) per k-block and
-    // commits once.
+  } else if (warp == kWarpXProducer) {
+    // ------------------------- activation producer --------------------------
+    // Activations may be the output of the previous kernel on the stream
+    // (programmatic dependent launch lets this kernel start while that one
+    // finishes): wait for it, then stream a stage's activation tiles into
+    // the slot whose MMAs have completed.
     if (lane == 0) {
+      griddep_wait();
       StageWalk w;
       walk_init(w, u0, u1, p);
-      int s = 0;
-      uint32_t k = 0;
+      Ring ra{0, 0};
       int64_t st = 0;
+      for (; w.u < u1; walk_next(w, u1, p), ++st, ring_next(ra, SA)) {
+        if (ra.use > 0 && !mbar_wait(&bars->aempty[ra.slot], (ra.use - 1) & 1, &bars->abort, p.status)) break;
+        uint8_t* dst = smem + p.x_base + static_cast<size_t>(ra.slot) * p.x_slot_bytes;
+        uint64_t* bar = &bars->xfull[ra.slot];
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(p.ks) * p.x_kb_bytes);
+        if (p.x3d) {
+          tma_load_3d(dst, &tm_x, 0, w.nt * p.ntile, w.kb, bar);
+        } else {
+          for (int j = 0; j < p.ks; ++j)
+            tma_load_2d(dst + j * p.x_kb_bytes, &tm_x, (w.kb + j) * 64, w.nt * p.ntile, bar);
+        }
+      }
+      for (int64_t q = st - SA > 0 ? st - SA : 0; q < st; ++q)
+        mbar_wait(&bars->xfull[q % SA], static_cast<uint32_t>(q / SA) & 1, nullptr, p.status);
+    }
+    __syncwarp();
+  } else if (warp >= kWarpMma && warp < kWarpMma + kMaxIssuers) {
+    // ----------------------------- MMA issuers ------------------------------
+    // Issuer i issues the MMAs of the k-blocks kb with kb % n_iss == i into
+    // its own accumulator; the epilogue adds the issuers' sums in a fixed
+    // order, so the result does not depend on the stage size or on timing.
+    // Per stage each issuer waits for the activation tiles and the rebuilt A
+    // tiles, issues 4 MMAs (K = 16 each) per k-block of its own and commits
+    // once (the slot is free when every issuer's commit has arrived).
+    const int iss = warp - kWarpMma;
+    if (lane == 0 && iss < p.n_iss) {
+      StageWalk w;
+      walk_init(w, u0, u1, p);
+      Ring ra{0, 0};
       uint32_t ab = 0;                 // accumulator buffer of this segment
-      uint32_t use_par[2] = {0u, 0u};  // completed-drain parity per buffer
-      uint32_t used[2] = {0u, 0u};     // segments already run per buffer
+      uint32_t use_par0 = 0u, use_par1 = 0u;  // completed-drain parity per buffer
+      uint32_t used0 = 0u, used1 = 0u;        // segments already run per buffer
       const uint32_t acc_stride = static_cast<uint32_t>(p.ntile);
-      const uint64_t b_desc0 = smem_desc_sw128(smem_u32(smem + p.off_x));
-      const uint64_t b_step = static_cast<uint64_t>(p.stage_bytes >> 4);
+      const uint64_t b_desc0 = smem_desc_sw128(smem_s + p.x_base);
+      const uint64_t b_step = static_cast<uint64_t>(p.x_slot_bytes >> 4);
       const uint64_t b_kb = static_cast<uint64_t>(p.x_kb_bytes >> 4);
-      bool first = true;
-      for (; w.u < u1; walk_next(w, u1, p), ++st) {
-        if (st > 0 && ++s == S) {
-          s = 0;
-          ++k;
-        }
+      bool seg_first = true;  // the next stage opens a segment
+      bool acc_zero = true;   // this issuer has not accumulated in the segment yet
+      for (; w.u < u1; walk_next(w, u1, p), ring_next(ra, SA)) {
         const bool last = (w.u + w.n == u1) || (w.kb + w.n == p.KB);
-        const uint32_t d_tmem = tmem + kAccCol + ab * acc_stride;
-        if (first && used[ab] > 0) {
-          if (!mbar_wait(&bars->acc_empty[ab], use_par[ab], &bars->abort, p.status)) break;
-          use_par[ab] ^= 1u;
-          tc_fence_after();
+        const uint32_t d_tmem = tmem + kAccCol + (ab * p.n_iss + iss) * acc_stride;
+        if (seg_first) {
+          const uint32_t used = ab ? used1 : used0;
+          if (used > 0) {
+            uint32_t& par = ab ? use_par1 : use_par0;
+            if (!mbar_wait(&bars->acc_empty[ab], par, &bars->abort, p.status)) break;
+            par ^= 1u;
+            tc_fence_after();
+          }
+          acc_zero = true;
         }
-        if (!mbar_wait(&bars->full[s], k & 1, &bars->abort, p.status)) break;
-        if (!mbar_wait(&bars->rebuilt[s], k & 1, &bars->abort, p.status)) break;
+        if (!mbar_wait(&bars->xfull[ra.slot], ra.use & 1, &bars->abort, p.status)) break;
+        if (!mbar_wait(&bars->afull[ra.slot], ra.use & 1, &bars->abort, p.status)) break;
         tc_fence_after();
-        const uint32_t a_tmem = tmem + p.a_col0 + static_cast<uint32_t>(s * p.ks) * 32;
-        const uint64_t b_desc = b_desc0 + static_cast<uint64_t>(s) * b_step;
+        const uint32_t a_tmem = tmem + p.a_col0 + static_cast<uint32_t>(ra.slot * p.ks) * 32;
+        const uint64_t b_desc = b_desc0 + static_cast<uint64_t>(ra.slot) * b_step;
         for (int j = 0; j < w.n; ++j) {
+          if ((w.kb + j) % p.n_iss != iss) continue;
           const uint32_t a = a_tmem + static_cast<uint32_t>(j) * 32;
           const uint64_t b = b_desc + static_cast<uint64_t>(j) * b_kb;
-          mma_ts(d_tmem, a + 0, b + 0, p.idesc, (first && j == 0) ? 0u : 1u);
+          mma_ts(d_tmem, a + 0, b + 0, p.idesc, acc_zero ? 0u : 1u);
           mma_ts(d_tmem, a + 8, b + 2, p.idesc, 1u);
           mma_ts(d_tmem, a + 16, b + 4, p.idesc, 1u);
           mma_ts(d_tmem, a + 24, b + 6, p.idesc, 1u);
+          acc_zero = false;
         }
-        tc_commit(&bars->empty[s]);
+        tc_commit(&bars->aempty[ra.slot]);
         if (last) {
           tc_commit(&bars->acc_full[ab]);
-          ++used[ab];
+          if (ab) ++used1;
+          else ++used0;
           if (p.n_acc == 2) ab ^= 1u;
         }
-        first = last;
+        seg_first = last;
       }
       // every MMA issued so far must finish before tensor memory is freed
-      tc_commit(&bars->drain);
-      mbar_wait(&bars->drain, 0, nullptr, p.status);
+      tc_commit(&bars->drain[iss]);
+      mbar_wait(&bars->drain[iss], 0, nullptr, p.status);
     }
     __syncwarp();
   } else if (warp < warp_epi0) {
@@ -730,21 +721,16 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + p.a_col0;
     StageWalk w;
     walk_init(w, u0, u1, p);
-    int s = 0;
-    uint32_t k = 0;
+    Ring rw{0, 0}, ra{0, 0};
     int turn = 0;  // stage index modulo G
-    for (int64_t st = 0; w.u < u1; walk_next(w, u1, p), ++st) {
-      if (st > 0) {
-        if (++s == S) {
-          s = 0;
-          ++k;
-        }
-        if (++turn == G) turn = 0;
-      }
+    for (int64_t st = 0; w.u < u1; walk_next(w, u1, p), ++st, ring_next(rw, SW), ring_next(ra, SA)) {
+      if (st > 0 && ++turn == G) turn = 0;
       if (turn != grp) continue;
-      if (!warp_wait(&bars->full[s], k & 1, bars, p.status)) break;
+      if (!warp_wait(&bars->wfull[rw.slot], rw.use & 1, bars, p.status)) break;
+      // the A slot is free once the MMAs of its previous use have completed
+      if (ra.use > 0 && !warp_wait(&bars->aempty[ra.slot], (ra.use - 1) & 1, bars, p.status)) break;
       tc_fence_after();
-      const uint32_t stage = smem_s + static_cast<uint32_t>(s) * p.stage_bytes;
+      const uint32_t stage = smem_s + p.w_base + static_cast<uint32_t>(rw.slot) * p.w_slot_bytes;
       int vbase = 0;  // pack: verbatim rows of the stage's earlier k-blocks
 #pragma unroll 1
       for (int j = 0; j < w.n; ++j) {
@@ -752,7 +738,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         rebuild_row<L>(stage, p, r, j, o);
         if constexpr (kPack) {
           // verbatim rows: one mask bit per row and k-block, no per-element test
-          const uint4 mk = lds128(stage + p.off_wa + j * kBody + kBodyMask);
+          const uint4 mk = lds128(stage + j * kBody + kBodyMask);
           const uint32_t m = mask_word(mk, q);
           if ((m >> lane) & 1) {
             const int idx = vbase + mask_below(mk, q) + __popc(m & ((1u << lane) - 1));
@@ -760,8 +746,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
               copy_row_s(stage + p.off_verb + idx * 128, o);
             } else {
               // more verbatim rows than staged ones: this one from HBM
-              const int64_t slot = static_cast<int64_t>(w.mt) * p.KB + w.kb - pt_min;
-              const long long g = static_cast<long long>(lds32(smem_s + p.soff_off + 4u * static_cast<uint32_t>(slot))) + idx;
+              const int64_t sl = static_cast<int64_t>(w.mt) * p.KB + w.kb - pt_min;
+              const long long g =
+                  static_cast<long long>(lds32(smem_s + p.soff_off + 4u * static_cast<uint32_t>(sl))) + idx;
               if (g < p.n_verbatim)
                 copy_row(reinterpret_cast<const uint4*>(p.tails + static_cast<uint64_t>(g) * 128u), o);
               else
@@ -789,23 +776,25 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             }
           }
         }
-        tmem_st32(lane_base + static_cast<uint32_t>(s * p.ks + j) * 32, o);
+        if (j == w.n - 1) {
+          // every read of the weight slot is done: hand it back to the producer
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars->wempty[rw.slot]);
+        }
+        tmem_st32(lane_base + static_cast<uint32_t>(ra.slot * p.ks + j) * 32, o);
       }
       tc_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->rebuilt[s]);
+      if (lane == 0) mbar_arrive(&bars->afull[ra.slot]);
     }
   } else {
     // ------------------------------- epilogue -------------------------------
     // the outputs, the gate operand and the workspace counters may still be
     // in use by the previous kernel on the stream until it has completed;
-    // tell the producer (activation loads) and let the next kernel launch
+    // then let the next kernel launch
     griddep_wait();
-    if (warp == warp_epi0 && lane == 0) {
-      st_release_cta(&bars->dep_ready, 1u);
-      griddep_launch_dependents();
-    }
+    if (warp == warp_epi0 && lane == 0) griddep_launch_dependents();
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const bool elected = warp == warp_epi0 && lane == 0;
@@ -855,6 +844,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       ++ch;
       return true;
     };
+    // the last contributor of a split tile to publish (elected thread) tells
+    // the others through this word
+    volatile uint32_t* last_flag = reinterpret_cast<volatile uint32_t*>(&bars->last_arriver);
     uint32_t seg = 0;
     int64_t u = u0;
     while (u < u1) {
@@ -865,18 +857,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       const int64_t c_first = unit_owner(t * p.KB, p);
       const int64_t c_last = unit_owner(t * p.KB + p.KB - 1, p);
       const int ncontrib = static_cast<int>(c_last - c_first + 1);
-      // A tile split over several CTAs is finished by the first of them
-      // (c_first): its part is the first k-blocks of the tile, the last
-      // segment of its range, so the other contributors (their parts open
-      // their ranges) have normally published long before.  It keeps its own
-      // sums in TMEM, adds the others' partials in CTA order and stores y.
-      // The others write partials and publish them with one release add.
-      const bool reducer = ncontrib > 1 && blockIdx.x == c_first;
-      const bool out_seg = ncontrib == 1 || reducer;
       const int b_first = nt * p.ntile;
       // output chunks past the batch are skipped (TMA would clip them anyway)
-      const int n_chunks = out_seg ? min(p.ntile, ((p.B - b_first + 15) / 16) * 16) / 16 : p.ntile / 16;
-      if (out_seg && tma_gate && elected && n_chunks > 0) load_gate(ch, mt, b_first);
+      const int n_chunks = min(p.ntile, ((p.B - b_first + 15) / 16) * 16) / 16;
+      if (ncontrib == 1 && tma_gate && elected && n_chunks > 0) load_gate(ch, mt, b_first);
       const uint32_t ab = seg % p.n_acc, use = seg / p.n_acc;
       bool ok = mbar_wait(&bars->acc_full[ab], use & 1, &bars->abort, p.status);
       ok = __all_sync(0xFFFFFFFFu, ok);
@@ -885,83 +869,96 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       tc_fence_after();
       const int64_t n = static_cast<int64_t>(mt) * 128 + r;
       const bool row_ok = n < p.N;
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + kAccCol + ab * static_cast<uint32_t>(p.ntile);
-      const int64_t slot0 = t + c_first;
-      bool staged = false;
-      if (reducer) {
-        bool got = true;
-        if (elected)
-          got = wait_count_at_least(p.counters + t, static_cast<uint32_t>(ncontrib - 1), &bars->abort, p.status,
-                                    kWaitLimitNs);
-        if (!group_and(got)) break;  // also orders the partial loads after the acquire
-        // on the CTA's last segment every stage has been consumed: copy the
-        // other partials of this thread's row into the stage buffers at once
-        // (one round trip), when they fit
-        staged = seg_end == u1 && static_cast<uint64_t>(S) * p.stage_bytes >=
-                                      static_cast<uint64_t>(ncontrib - 1) * 512u * static_cast<uint32_t>(p.ntile);
-        if (staged) {
-          float* stg = reinterpret_cast<float*>(smem);
-          for (int jc = 1; jc < ncontrib; ++jc) {
-            const float* src = p.partials + ((slot0 + jc) * 128 + r) * p.ntile;
-            float* dst = stg + (static_cast<size_t>(jc - 1) * 128 + r) * p.ntile;
-            for (int f = 0; f < n_chunks * 16; f += 4) cp_async_16(dst + f, src + f);
-          }
-          cp_async_wait_all();
+      const uint32_t taddr =
+          tmem + (static_cast<uint32_t>(q * 32) << 16) + kAccCol + ab * p.n_iss * static_cast<uint32_t>(p.ntile);
+      // issuers that accumulated in this segment: issuer i took the
+      // k-blocks kb % n_iss == i, so a segment shorter than n_iss k-blocks
+      // leaves some without any
+      const int kb_first = static_cast<int>(u - t * p.KB);
+      const int n_seg = static_cast<int>(seg_end - u);
+      uint32_t active = 0;  // bit i: issuer i accumulated
+      for (int d = 0; d < p.n_iss && d < n_seg; ++d) active |= 1u << ((kb_first + d) % p.n_iss);
+      // this CTA's sum of 16 columns: the issuers' sums added in issuer
+      // order (0, 1, 2, 3), skipping issuers without k-blocks
+      auto own_sum = [&](int cc, float (&acc)[16]) {
+        bool have = false;
+        for (int i = 0; i < p.n_iss; ++i) {
+          if (!((active >> i) & 1)) continue;
+          uint32_t v[16];
+          tmem_ld16(taddr + static_cast<uint32_t>(i * p.ntile) + cc * 16, v);
+          tc_wait_ld();
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) acc[jj] = have ? acc[jj] + __uint_as_float(v[jj]) : __uint_as_float(v[jj]);
+          have = true;
         }
-      }
-      float* my_part = p.partials + ((slot0 + (blockIdx.x - c_first)) * 128 + r) * p.ntile;
-      for (int cc = 0; cc < n_chunks && ok; ++cc) {
-        uint32_t v[16];
-        tmem_ld16(taddr + cc * 16, v);
-        tc_wait_ld();
-        if (!out_seg) {
+      };
+      if (ncontrib == 1) {
+        for (int cc = 0; cc < n_chunks && ok; ++cc) {
+          float acc[16];
+          own_sum(cc, acc);
+          if (!emit(acc, mt, b_first + cc * 16, n, row_ok)) {
+            ok = false;
+            break;
+          }
+          if (tma_gate && elected && cc + 1 < n_chunks) load_gate(ch, mt, b_first + (cc + 1) * 16);
+        }
+        if (!ok) break;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);
+      } else {
+        // A tile split over several CTAs (stream-K): every contributor
+        // writes its sum to its partial slot and takes a ticket; the last to
+        // arrive adds all partials in CTA order and stores y.  Nobody waits
+        // for another CTA, and the sum is the same whoever finishes last.
+        const int64_t slot0 = t + c_first;
+        float* my_part = p.partials + ((slot0 + (blockIdx.x - c_first)) * 128 + r) * p.ntile;
+        for (int cc = 0; cc < n_chunks; ++cc) {
+          float acc[16];
+          own_sum(cc, acc);
           float4* dst = reinterpret_cast<float4*>(my_part + cc * 16);
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4)
-            dst[q4] = make_float4(__uint_as_float(v[4 * q4]), __uint_as_float(v[4 * q4 + 1]),
-                                  __uint_as_float(v[4 * q4 + 2]), __uint_as_float(v[4 * q4 + 3]));
-          continue;
+            dst[q4] = make_float4(acc[4 * q4], acc[4 * q4 + 1], acc[4 * q4 + 2], acc[4 * q4 + 3]);
         }
-        float acc[16];
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) acc[jj] = __uint_as_float(v[jj]);
-        if (reducer) {
-          // the other contributors' partials of these 16 columns, CTA order
-          for (int jc = 1; jc < ncontrib; ++jc) {
-            const float4* src =
-                staged ? reinterpret_cast<const float4*>(reinterpret_cast<const float*>(smem) +
-                                                         (static_cast<size_t>(jc - 1) * 128 + r) * p.ntile + cc * 16)
-                       : reinterpret_cast<const float4*>(p.partials + ((slot0 + jc) * 128 + r) * p.ntile + cc * 16);
-            float4 w4[4];
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) w4[q4] = staged ? src[q4] : __ldcg(src + q4);
-#pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
-              acc[4 * q4] += w4[q4].x;
-              acc[4 * q4 + 1] += w4[q4].y;
-              acc[4 * q4 + 2] += w4[q4].z;
-              acc[4 * q4 + 3] += w4[q4].w;
-            }
-          }
-        }
-        if (!emit(acc, mt, b_first + cc * 16, n, row_ok)) {
-          ok = false;
-          break;
-        }
-        if (tma_gate && elected && cc + 1 < n_chunks) load_gate(ch, mt, b_first + (cc + 1) * 16);
-      }
-      if (!ok) break;
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);
-      if (ncontrib > 1) {
-        group_sync();  // every partial store of the group precedes the publish
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);
+        group_sync();  // every partial store of the group precedes the ticket
         if (elected) {
-          if (reducer)
-            p.counters[t] = 0;  // ready for the next launch on this workspace
-          else
-            red_release_gpu_add(p.counters + t, 1u);
+          const uint32_t before = atom_add_acq_rel_gpu(p.counters + t, 1u);
+          const bool last = before == static_cast<uint32_t>(ncontrib - 1);
+          if (last) p.counters[t] = 0;  // every contributor has arrived: ready for the next launch
+          *last_flag = last ? 1u : 0u;
         }
+        group_sync();  // the flag, and the acquired partials, for the whole group
+        if (*last_flag) {
+          if (tma_gate && elected && n_chunks > 0) load_gate(ch, mt, b_first);
+          for (int cc = 0; cc < n_chunks && ok; ++cc) {
+            float acc[16];
+            for (int jc = 0; jc < ncontrib; ++jc) {
+              const float4* src =
+                  reinterpret_cast<const float4*>(p.partials + ((slot0 + jc) * 128 + r) * p.ntile + cc * 16);
+              float4 w4[4];
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) w4[q4] = __ldcg(src + q4);
+#pragma unroll
+              for (int q4 = 0; q4 < 4; ++q4) {
+                acc[4 * q4] = jc ? acc[4 * q4] + w4[q4].x : w4[q4].x;
+                acc[4 * q4 + 1] = jc ? acc[4 * q4 + 1] + w4[q4].y : w4[q4].y;
+                acc[4 * q4 + 2] = jc ? acc[4 * q4 + 2] + w4[q4].z : w4[q4].z;
+                acc[4 * q4 + 3] = jc ? acc[4 * q4 + 3] + w4[q4].w : w4[q4].w;
+              }
+            }
+            if (!emit(acc, mt, b_first + cc * 16, n, row_ok)) {
+              ok = false;
+              break;
+            }
+            if (tma_gate && elected && cc + 1 < n_chunks) load_gate(ch, mt, b_first + (cc + 1) * 16);
+          }
+          if (!ok) break;
+        }
+        group_sync();  // the flag word is reused by the next split segment
       }
       ++seg;
       u = seg_end;
@@ -970,7 +967,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     // chunks still in flight after an abort, and the output stores
     if (elected && tma_gate)
       for (uint32_t c = ch; c < gate_next; ++c) mbar_wait(&bars->gate_full[c & 1], (c >> 1) & 1, nullptr, p.status);
-    if (elected && p.tma_out) bulk_wait_group0();
+    if (elected && p.tma_out) bulk_wait_group_read0();
   }
 
   tc_fence_before();
@@ -991,8 +988,9 @@ __global__ void swiglu_kernel(const __nv_bfloat16* __restrict__ g, const __nv_bf
 // ------------------------------ host side ------------------------------------
 
 struct Layout {
-  int stages = 0, ks = 1, groups = 1;
-  uint32_t stage_bytes = 0, off_x = 0, off_wa = 0, off_wb = 0, off_verb = 0, off_hdr = 0;
+  int sw = 0, sa = 0, ks = 1, groups = 1, n_iss = 1, n_acc = 1;
+  uint32_t w_slot_bytes = 0, x_slot_bytes = 0, w_base = 0, x_base = 0, ring_bytes = 0;
+  uint32_t off_wb = 0, off_verb = 0, off_hdr = 0;
   uint32_t x_kb_bytes = 0;
   uint32_t meta_off = 0, meta_slot_words = 0, bar_off = 0, soff_off = 0, a_col0 = 0, epi_off = 0;
   int n_soff = 0, vcap = 0;
@@ -1007,9 +1005,9 @@ int env_int(const char* name, int dflt, int lo, int hi) {
   return x < lo ? lo : (x > hi ? hi : x);
 }
 
-// Pipeline depth cap (UW_MAX_STAGES overrides, for tuning).
-int max_stages() {
-  static int v = env_int("UW_MAX_STAGES", kMaxStages, 2, kMaxStages);
+// Ring depth cap (UW_MAX_STAGES overrides, for tuning).
+int max_slots() {
+  static int v = env_int("UW_MAX_STAGES", kMaxSlots, 2, kMaxSlots);
   return v;
 }
 
@@ -1021,49 +1019,61 @@ int rebuild_groups() {
 
 // k-blocks per stage: several for small batch tiles, where the per-stage
 // costs dominate; one when the activation tile is large (UW_STAGE_KBLOCKS
-// overrides, for tuning).
+// overrides, for tuning).  The stage size does not change any result.
 int stage_kblocks(int loader, int ntile, int KB) {
   static int forced = env_int("UW_STAGE_KBLOCKS", 0, 0, kMaxKS);
   int ks;
   if (loader_idx4(loader)) ks = 1;
   else if (forced) ks = forced;
-  else if (loader == kBF16) ks = ntile <= 32 ? 2 : 1;
+  else if (ntile <= 16) ks = 3;
   else ks = ntile <= 64 ? 2 : 1;
   return std::max(1, std::min(ks, KB));
 }
 
-// Shared-memory plan of one launch.  Every tile region starts on a 1024-byte
-// boundary (the 128-byte swizzle of the activation tile repeats every 1024).
+// Shared-memory and tensor-memory plan of one launch.  Every tile region
+// starts on a 1024-byte boundary (the 128-byte swizzle of the activation
+// tile repeats every 1024 bytes).
+bool make_layout_ks(int loader, const GemmPlan& plan, int wpr, bool tma_out, bool gate, int ks_want, Layout* out);
+
 bool make_layout(int loader, const GemmPlan& plan, int wpr, bool tma_out, bool gate, Layout* out) {
+  // the preferred stage size, else smaller ones when it does not fit
+  for (int ks = stage_kblocks(loader, plan.ntile, plan.KB); ks >= 1; --ks)
+    if (make_layout_ks(loader, plan, wpr, tma_out, gate, ks, out)) return true;
+  return false;
+}
+
+bool make_layout_ks(int loader, const GemmPlan& plan, int wpr, bool tma_out, bool gate, int ks_want, Layout* out) {
   Layout l;
-  l.ks = stage_kblocks(loader, plan.ntile, plan.KB);
+  l.ks = ks_want;
   const uint32_t ks = static_cast<uint32_t>(l.ks);
-  // TMEM: accumulators (n_acc x ntile columns), then 32 columns of rebuilt A
-  // per k-block of every stage
-  const int n_acc = 2 * plan.ntile <= 256 ? 2 : 1;
-  l.a_col0 = (static_cast<uint32_t>(n_acc * plan.ntile) + 31u) & ~31u;
-  const int tmem_stages = static_cast<int>((kTmemCols - l.a_col0) / (32u * ks));
+  // TMEM: accumulators (n_acc buffers x n_iss issuers x ntile columns), then
+  // 32 columns of rebuilt A per k-block of every activation slot.  Two
+  // issuers (each summing its own k-blocks) when their accumulators leave
+  // half of tensor memory to the A tiles.  The issuer count depends only on
+  // the batch tile, so every pipeline sums in the same order.
+  l.n_acc = 2 * plan.ntile <= 256 ? 2 : 1;
+  l.n_iss = l.n_acc * 4 * plan.ntile <= 256 ? 4 : (l.n_acc * 2 * plan.ntile <= 256 ? 2 : 1);
+  l.a_col0 = (static_cast<uint32_t>(l.n_acc * l.n_iss * plan.ntile) + 31u) & ~31u;
+  const int tmem_slots = static_cast<int>((kTmemCols - l.a_col0) / (32u * ks));
   l.x_kb_bytes = static_cast<uint32_t>(plan.ntile) * 128;
+  l.x_slot_bytes = ks * l.x_kb_bytes;  // a multiple of 2048
   const bool idx4 = loader_idx4(loader);
   const bool pack = loader_pack(loader);
-  l.off_x = 0;
-  l.off_wa = a1024(ks * l.x_kb_bytes);
+  uint32_t w_min = 0;
   if (pack) {
-    l.off_wb = l.off_wa + kBodyIdx;  // unused: indices are inside each body
-    l.off_verb = (l.off_wa + ks * kBody + 127u) & ~127u;
-    l.stage_bytes = a1024(l.off_verb + kPackMinTail * 128u);
+    l.off_verb = (ks * kBody + 127u) & ~127u;
+    w_min = a1024(l.off_verb + kPackMinTail * 128u);
   } else if (loader == kBF16) {
-    l.off_wb = l.off_wa;
-    l.stage_bytes = l.off_wa + ks * 16384u;
+    w_min = ks * 16384u;
   } else if (loader == kEXP8) {
-    l.off_wb = l.off_wa + ks * 8192u;
-    l.stage_bytes = l.off_wb + ks * 8192u;
+    l.off_wb = ks * 8192u;
+    w_min = l.off_wb + ks * 8192u;
   } else {
-    l.off_wb = l.off_wa + ks * 8192u;
+    l.off_wb = ks * 8192u;
     l.off_verb = a1024(l.off_wb + ks * 4096u);
     l.off_hdr = l.off_verb + kVCap * 128u;
     l.vcap = kVCap;
-    l.stage_bytes = a1024(l.off_hdr + 64u);
+    w_min = a1024(l.off_hdr + 64u);
   }
   l.meta_slot_words = idx4 ? 128u * static_cast<uint32_t>(wpr) : 0u;
   const uint32_t meta_bytes = a1024(2u * 2u * l.meta_slot_words * 4u);
@@ -1080,29 +1090,42 @@ bool make_layout(int loader, const GemmPlan& plan, int wpr, bool tma_out, bool g
   const uint32_t epi_bytes = tma_out ? (gate ? 16384u : 8192u) : 0u;
   const uint32_t fixed = meta_bytes + soff_bytes + epi_bytes + a1024(sizeof(Bars)) + 1024u;  // + alignment slack
   if (fixed >= kSmemLimit) return false;
-  int stages = static_cast<int>((kSmemLimit - fixed) / l.stage_bytes);
-  stages = std::min({stages, max_stages(), tmem_stages});
-  if (stages < 2) return false;
+  const uint32_t room = static_cast<uint32_t>(kSmemLimit) - fixed;
   // Rebuild group g takes the stages i with i % groups == g.  A group may
   // only wait for a ring slot's next phase once its current phase has
   // completed (the wait tests a phase parity), which holds when every slot
-  // always belongs to the same group: stages must be a multiple of groups.
-  l.groups = std::min(rebuild_groups(), stages);
-  stages -= stages % l.groups;
-  l.stages = stages;
+  // of both rings always belongs to the same group: slot counts are
+  // multiples of groups.
+  // activation ring: as deep as tensor memory allows (its slots are cheap
+  // at small batch), within half of the shared memory
+  int sa = std::min({tmem_slots, max_slots(), static_cast<int>((room / 2) / l.x_slot_bytes)});
+  if (sa < 2) return false;
+  l.groups = std::min(rebuild_groups(), sa);
+  sa -= sa % l.groups;
+  const uint32_t w_room = room - static_cast<uint32_t>(sa) * l.x_slot_bytes;
+  int sw = std::min(static_cast<int>(w_room / w_min), max_slots());
+  sw -= sw % l.groups;
+  if (sw < l.groups || sw < 2) return false;
+  l.sa = sa;
+  l.sw = sw;
+  l.x_base = 0;
+  l.w_base = static_cast<uint32_t>(sa) * l.x_slot_bytes;
+  l.w_slot_bytes = w_min;
   if (pack) {
-    // spread the remaining shared memory over the stages as on-chip verbatim
-    // rows (most tiles have a few; the rest come from HBM)
-    const uint32_t per_stage = ((kSmemLimit - fixed) / static_cast<uint32_t>(stages)) & ~1023u;
-    const uint32_t room = (per_stage - l.off_verb) / 128u;
-    l.vcap = static_cast<int>(std::min<uint32_t>(room, 128u * ks));
-    l.stage_bytes = a1024(l.off_verb + static_cast<uint32_t>(l.vcap) * 128u);
+    // spread the remaining shared memory over the weight slots as on-chip
+    // verbatim rows (most tiles have a few; the rest come from HBM)
+    const uint32_t per_slot = (w_room / static_cast<uint32_t>(sw)) & ~1023u;
+    const uint32_t rows = (per_slot - l.off_verb) / 128u;
+    l.vcap = static_cast<int>(std::min<uint32_t>(rows, 128u * ks));
+    l.w_slot_bytes = a1024(l.off_verb + static_cast<uint32_t>(l.vcap) * 128u);
   }
-  l.meta_off = static_cast<uint32_t>(stages) * l.stage_bytes;
+  l.ring_bytes = l.w_base + static_cast<uint32_t>(sw) * l.w_slot_bytes;
+  l.meta_off = l.ring_bytes;
   l.soff_off = l.meta_off + meta_bytes;
   l.epi_off = l.soff_off + soff_bytes;
   l.bar_off = l.epi_off + epi_bytes;
   l.smem = std::max<size_t>(static_cast<size_t>(l.bar_off) + a1024(sizeof(Bars)) + 1024u, kSmemFloor);
+  if (l.smem > kSmemLimit + 1024u) return false;
   *out = l;
   return true;
 }
@@ -1125,7 +1148,7 @@ uw_status launch_kernel(const CUtensorMap& x, const CUtensorMap& wa, const CUten
   // outputs
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(kp.grid));
-  cfg.blockDim = dim3(static_cast<unsigned>(32 * (6 + 4 * kp.groups)));
+  cfg.blockDim = dim3(static_cast<unsigned>(32 * (10 + 4 * kp.groups)));
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -1256,11 +1279,14 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.ntile = plan.ntile;
   kp.units = plan.units;
   kp.grid = plan.grid;
-  kp.stages = lay.stages;
   kp.ks = lay.ks;
-  kp.stage_bytes = lay.stage_bytes;
-  kp.off_x = lay.off_x;
-  kp.off_wa = lay.off_wa;
+  kp.sw = lay.sw;
+  kp.sa = lay.sa;
+  kp.n_iss = lay.n_iss;
+  kp.w_slot_bytes = lay.w_slot_bytes;
+  kp.x_slot_bytes = lay.x_slot_bytes;
+  kp.w_base = lay.w_base;
+  kp.x_base = lay.x_base;
   kp.off_wb = lay.off_wb;
   kp.off_verb = lay.off_verb;
   kp.off_hdr = lay.off_hdr;
@@ -1283,7 +1309,7 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.idesc = idesc_bf16_f32(plan.ntile);
   kp.groups = lay.groups;
   kp.vcap = lay.vcap;
-  kp.n_acc = 2 * plan.ntile <= 256 ? 2 : 1;
+  kp.n_acc = lay.n_acc;
   kp.pack = a.pack;
   kp.tails = a.pack ? a.pack + static_cast<uint64_t>(plan.n_mtiles) * plan.KB * kBody : nullptr;
   kp.pack_off = a.pack_off;
