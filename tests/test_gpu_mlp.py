@@ -30,7 +30,7 @@ def _block(d, ffn, seed):
     return gate, up, down
 
 
-@pytest.mark.parametrize("B", [1, 8, 33])
+@pytest.mark.parametrize("B", [1, 8, 33, 100, 200])
 def test_mlp_block_small(B):
     gate, up, down = _block(512, 1536, 61)
     dms = [device_matrix(m) for m in (gate, up, down)]
@@ -63,6 +63,30 @@ def test_fused_swiglu_epilogue_equals_separate_kernels():
     uw.gemm_direct_palette(dms[2], h, y2, ws)
     ws.check()
     assert np.array_equal(to_host_u16(y), to_host_u16(y2))
+
+
+@pytest.mark.parametrize("B", [4, 40])
+def test_block_with_heavy_verbatim_and_ragged_rows(B):
+    """Direct-palette block whose gate and up tiles carry many verbatim rows
+    (some beyond the rows staged on chip) and whose hidden size (1088) leaves
+    a partial last row tile.  It must equal the exponent-only pipeline bit
+    for bit and meet the MLP bar against the float64 oracle."""
+    d, ffn = 512, 1088
+    gate = synth.weight_matrix(ffn, d, 0.02, 2e-2, 300.0, 67)
+    up = synth.weight_matrix(ffn, d, 0.02, 2e-2, 300.0, 68)
+    down = synth.weight_matrix(d, ffn, 0.02, 1e-3, 100.0, 69)
+    dms = [device_matrix(m) for m in (gate, up, down)]
+    x = synth.activations(B, d, 70)
+    outs = []
+    for pipes in ([3, 3, 3], [1, 1, 3]):
+        ws = uw.Workspace(uw.mlp_workspace_bytes(*dms, pipes, B))
+        y = empty_bf16(B, d)
+        uw.mlp_block(*dms, pipes, to_dev(x), y, ws)
+        ws.check("mlp")
+        outs.append(to_host_u16(y))
+    assert np.array_equal(outs[0], outs[1])
+    ok, err, rms = mlp_check(outs[0], gate, up, down, x)
+    assert ok, (err, rms)
 
 
 def test_full_size_mlp_block_batch8():
