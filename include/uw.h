@@ -238,9 +238,12 @@ UW_API uw_status uw_validate(const uw_matrix* host_mirror);
 /* Bytes of device workspace (library plumbing; no counterpart on the page)
  * a device call needs for this matrix, pipeline and batch (batch 0 for the
  * decode/transcode calls).  The workspace holds a
- * status word, split-K partial sums and tile counters, and for the FULL /
- * EXPONENT / TRANSCODE pipelines the intermediate decoded matrix.  Returns 0
- * for invalid arguments. */
+ * 256-byte header (status word), a fixed 64 KB region of split-K tile
+ * counters, the split-K partial sums, and for the FULL / EXPONENT /
+ * TRANSCODE pipelines the intermediate decoded matrix.  The regions start
+ * at the same offsets for every matrix and batch, so calls on different
+ * matrices may share one workspace of the largest size they need.  Returns
+ * 0 for invalid arguments. */
 UW_API size_t uw_workspace_bytes(const uw_layout* L, int32_t pipeline, int32_t batch);
 
 /* Zero a workspace and record its size in its header (library plumbing;
@@ -333,8 +336,10 @@ UW_API uw_status uw_pack_direct_palette(const uw_matrix* m, const uint32_t* pack
  * m->pack and m->pack_off must be set (uw_pack_direct_palette).  The split of the K
  * loop across CTAs and the order of its reduction depend only on (rows, cols,
  * batch, SM count), so all pipelines give bit-identical y.
- * batch: 1..512.  Errors: UW_ERR_INVALID_ARG, UW_ERR_UNSUPPORTED_SHAPE,
- * UW_ERR_WORKSPACE_TOO_SMALL, UW_ERR_CUDA. */
+ * batch: 1..512; cols <= 32768; ceil(rows/128) * ceil(batch/256) <= 16384
+ * output tiles (rows <= 2097152 up to batch 256).  Errors:
+ * UW_ERR_INVALID_ARG, UW_ERR_UNSUPPORTED_SHAPE, UW_ERR_WORKSPACE_TOO_SMALL,
+ * UW_ERR_CUDA. */
 UW_API uw_status uw_gemm_direct_palette(const uw_matrix* m, const uint16_t* x, int32_t batch,
                                  uint16_t* y, void* workspace, size_t workspace_bytes,
                                  void* stream);
@@ -366,8 +371,8 @@ UW_API uw_status uw_gemm_direct_palette_general_lookup(const uw_matrix* m, const
  * (no cudaMalloc/cudaFree, no allocating library call).
  *   - Every GPU that loads the library holds that 16 MiB until exit.
  *   - Limit: header + tile counters + split-K partials must fit in it, i.e.
- *     (ceil(rows/128)*ceil(batch/256) + SMs) * batch_tile * 512 bytes plus a
- *     few KB, batch_tile = batch rounded up to a multiple of 16 (per 256);
+ *     (ceil(rows/128)*ceil(batch/256) + SMs) * batch_tile * 512 bytes plus
+ *     64.25 KB, batch_tile = batch rounded up to a multiple of 16 (per 256);
  *     on a 148-SM B200 a 14336 x 4096 matrix fits up to batch 112.  Larger
  *     sizes return UW_ERR_WORKSPACE_TOO_SMALL before anything is launched.
  *   - The first call on a device looks the array's device address up
@@ -415,6 +420,29 @@ UW_API size_t uw_mlp_workspace_bytes(const uw_matrix* gate, const uw_matrix* up,
 UW_API uw_status uw_mlp_block(const uw_matrix* gate, const uw_matrix* up, const uw_matrix* down,
                        const int32_t* pipelines, const uint16_t* x, int32_t batch, uint16_t* y,
                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* The MLP part of one decode step through an n_layers stack (section "Why
+ * compression is harder than it looks": per-token latency adds up over every
+ * layer's matrices): h_0 = x, h_{l+1} = MLP_l(h_l) with MLP_l the block of
+ * uw_mlp_block over mats[3l], mats[3l+1], mats[3l+2] (gate, up, down) and
+ * pipelines[3l..3l+2]; y = h_{n_layers}.  Attention and residual paths are
+ * not part of it: each layer's MLP output is the next layer's input, which
+ * keeps the dependency between layers.  Every layer maps d -> d (the same
+ * d; ffn may differ).  x, y: device BF16 [batch, d]; mats: host array of
+ * 3*n_layers pointers.  All 3*n_layers GEMMs (with the decoders their
+ * pipelines need) go onto `stream` back to back; each GEMM may start
+ * streaming its weights while the one before it finishes (programmatic
+ * dependent launch).  Nothing synchronizes.  Workspace:
+ * uw_mlp_stack_workspace_bytes (0 for invalid arguments): the largest
+ * block's workspace plus two [batch, d] activation buffers.  Errors:
+ * UW_ERR_INVALID_ARG (NULL pointers, n_layers < 1, shapes that do not
+ * chain), UW_ERR_WORKSPACE_TOO_SMALL, and the errors of uw_mlp_block; on an
+ * error the layers before it are already enqueued. */
+UW_API size_t uw_mlp_stack_workspace_bytes(const uw_matrix* const* mats, const int32_t* pipelines,
+                                           int32_t n_layers, int32_t batch);
+UW_API uw_status uw_mlp_stack(const uw_matrix* const* mats, const int32_t* pipelines, int32_t n_layers,
+                              const uint16_t* x, int32_t batch, uint16_t* y, void* workspace,
+                              size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Autotuner (sections "Key Points" and "Why no single pipeline wins")

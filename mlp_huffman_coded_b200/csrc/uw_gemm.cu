@@ -964,10 +964,14 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       u = seg_end;
     }
     // the CTA's shared memory must outlive the copies touching it: gate
-    // chunks still in flight after an abort, and the output stores
+    // chunks still in flight after an abort.  The output stores must have
+    // completed, not only read shared memory: the next kernel on the stream
+    // may read y as soon as this grid has exited (programmatic dependent
+    // launch), and a layer's input read right away raced with stores still
+    // in flight
     if (elected && tma_gate)
       for (uint32_t c = ch; c < gate_next; ++c) mbar_wait(&bars->gate_full[c & 1], (c >> 1) & 1, nullptr, p.status);
-    if (elected && p.tma_out) bulk_wait_group_read0();
+    if (elected && p.tma_out) bulk_wait_group0();
   }
 
   tc_fence_before();
@@ -1500,14 +1504,11 @@ extern "C" size_t uw_mlp_workspace_bytes(const uw_matrix* gate, const uw_matrix*
   return mlp_ws(gate, up, down, pipelines, batch, &w) ? w.total : 0;
 }
 
-extern "C" uw_status uw_mlp_block(const uw_matrix* gate, const uw_matrix* up, const uw_matrix* down,
-                                  const int32_t* pipelines, const uint16_t* x, int32_t batch, uint16_t* y,
-                                  void* ws, size_t ws_bytes, void* stream) {
-  MlpWs w;
-  if (!ws || !x || !y) return UW_ERR_INVALID_ARG;
-  if (!mlp_ws(gate, up, down, pipelines, batch, &w)) return UW_ERR_INVALID_ARG;
-  if (ws_bytes < w.total) return UW_ERR_WORKSPACE_TOO_SMALL;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+namespace {
+// One block on the stream: g = x Wg^T, h = SiLU(g) * (x Wu^T) (fused into
+// the up GEMM's epilogue), y = h Wd^T.  `w` sizes the workspace regions.
+uw_status run_block(const uw_matrix* gate, const uw_matrix* up, const uw_matrix* down, const int32_t* pipelines,
+                    const uint16_t* x, int32_t batch, uint16_t* y, void* ws, const MlpWs& w, cudaStream_t s) {
   uint8_t* base = static_cast<uint8_t*>(ws);
   void* scratch = base + w.gemm;
   uint16_t* g = reinterpret_cast<uint16_t*>(base + w.gemm + w.scratch);
@@ -1517,4 +1518,70 @@ extern "C" uw_status uw_mlp_block(const uw_matrix* gate, const uw_matrix* up, co
   st = run_pipeline(up, pipelines[1], x, batch, h, g, ws, w.gemm, scratch, w.scratch, s);
   if (st != UW_OK) return st;
   return run_pipeline(down, pipelines[2], h, batch, y, nullptr, ws, w.gemm, scratch, w.scratch, s);
+}
+
+// Workspace of an n-layer stack: the largest block's regions, then two
+// activation buffers [batch, d] that the layers' outputs alternate between.
+struct StackWs {
+  MlpWs blk;
+  size_t act = 0, total = 0;
+};
+bool stack_ws(const uw_matrix* const* mats, const int32_t* pipes, int32_t n_layers, int32_t batch, StackWs* out) {
+  if (!mats || !pipes || n_layers < 1) return false;
+  StackWs sw;
+  int64_t d = -1;
+  for (int32_t l = 0; l < n_layers; ++l) {
+    MlpWs w;
+    if (!mlp_ws(mats[3 * l], mats[3 * l + 1], mats[3 * l + 2], pipes + 3 * l, batch, &w)) return false;
+    const int64_t dl = mats[3 * l]->L.cols;
+    if (d >= 0 && dl != d) return false;  // every layer maps d -> d
+    d = dl;
+    sw.blk.gemm = std::max(sw.blk.gemm, w.gemm);
+    sw.blk.scratch = std::max(sw.blk.scratch, w.scratch);
+    sw.blk.gbuf = std::max(sw.blk.gbuf, w.gbuf);
+    sw.blk.hbuf = std::max(sw.blk.hbuf, w.hbuf);
+  }
+  sw.blk.total = sw.blk.gemm + sw.blk.scratch + sw.blk.gbuf + sw.blk.hbuf;
+  sw.act = n_layers > 1 ? align_up(static_cast<size_t>(batch) * d * 2, 256) : 0;
+  sw.total = sw.blk.total + 2 * sw.act;
+  *out = sw;
+  return true;
+}
+}  // namespace
+
+extern "C" uw_status uw_mlp_block(const uw_matrix* gate, const uw_matrix* up, const uw_matrix* down,
+                                  const int32_t* pipelines, const uint16_t* x, int32_t batch, uint16_t* y,
+                                  void* ws, size_t ws_bytes, void* stream) {
+  MlpWs w;
+  if (!ws || !x || !y) return UW_ERR_INVALID_ARG;
+  if (!mlp_ws(gate, up, down, pipelines, batch, &w)) return UW_ERR_INVALID_ARG;
+  if (ws_bytes < w.total) return UW_ERR_WORKSPACE_TOO_SMALL;
+  return run_block(gate, up, down, pipelines, x, batch, y, ws, w, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t uw_mlp_stack_workspace_bytes(const uw_matrix* const* mats, const int32_t* pipelines,
+                                               int32_t n_layers, int32_t batch) {
+  StackWs w;
+  return stack_ws(mats, pipelines, n_layers, batch, &w) ? w.total : 0;
+}
+
+extern "C" uw_status uw_mlp_stack(const uw_matrix* const* mats, const int32_t* pipelines, int32_t n_layers,
+                                  const uint16_t* x, int32_t batch, uint16_t* y, void* ws, size_t ws_bytes,
+                                  void* stream) {
+  StackWs w;
+  if (!ws || !x || !y) return UW_ERR_INVALID_ARG;
+  if (!stack_ws(mats, pipelines, n_layers, batch, &w)) return UW_ERR_INVALID_ARG;
+  if (ws_bytes < w.total) return UW_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint16_t* act[2] = {reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + w.blk.total),
+                      reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + w.blk.total + w.act)};
+  const uint16_t* in = x;
+  for (int32_t l = 0; l < n_layers; ++l) {
+    uint16_t* out = l == n_layers - 1 ? y : act[l & 1];
+    const uw_status st =
+        run_block(mats[3 * l], mats[3 * l + 1], mats[3 * l + 2], pipelines + 3 * l, in, batch, out, ws, w.blk, s);
+    if (st != UW_OK) return st;
+    in = out;
+  }
+  return UW_OK;
 }

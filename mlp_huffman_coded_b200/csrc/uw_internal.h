@@ -40,6 +40,11 @@ uw_status make_tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const 
 // Workspace layout: [0, 256) header (status word at offset 0), then tile
 // counters, split-K partials and the pipeline's intermediate matrix.
 constexpr size_t kWsHeader = 256;
+// Split-K tile counters: one fixed-size region right after the header, so
+// the partial sums start at the same offset for every GEMM plan and one
+// GEMM's partials never land on another's counters when calls share a
+// workspace.  16384 tiles.
+constexpr size_t kCounterBytes = 64 * 1024;
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 // Shape of one GEMM launch, shared by every pipeline so that the K split and

@@ -124,7 +124,8 @@ uw_status gemm_plan(int64_t N, int64_t K, int B, int sm_count, GemmPlan* out) {
   p.units = static_cast<int64_t>(p.n_mtiles) * p.n_ntiles * p.KB;
   p.grid = static_cast<int>(p.units < sm_count ? p.units : sm_count);
   const int64_t n_tiles = static_cast<int64_t>(p.n_mtiles) * p.n_ntiles;
-  p.counter_bytes = align_up(static_cast<size_t>(n_tiles) * 4, 256);
+  if (static_cast<size_t>(n_tiles) * 4 > kCounterBytes) return UW_ERR_UNSUPPORTED_SHAPE;
+  p.counter_bytes = kCounterBytes;
   p.partial_bytes = static_cast<size_t>(n_tiles + p.grid) * p.ntile * 128 * 4;
   *out = p;
   return UW_OK;

@@ -23,6 +23,7 @@ __all__ = [
     "WORKLOADS",
     "stack_sigmas",
     "stack_layer",
+    "stack_layer_device",
 ]
 
 
@@ -118,6 +119,29 @@ def stack_layer(layer: int, n_layers: int = 32, d_model: int = 4096, ffn: int = 
     return (weight_matrix(ffn, d_model, sigma, outlier_rate, outlier_scale, seed),
             weight_matrix(ffn, d_model, sigma, outlier_rate, outlier_scale, seed + 1),
             weight_matrix(d_model, ffn, sigma, outlier_rate, outlier_scale, seed + 2))
+
+
+def stack_layer_device(layer: int, device, n_layers: int = 32, d_model: int = 4096, ffn: int = 14336,
+                       outlier_rate: float = 1e-3, outlier_scale: float = 100.0):
+    """Layer `layer` of the 32-layer stack drawn on a torch device: the recipe
+    of `stack_layer` (the layer's sigma, N(0, sigma) weights, outliers at
+    `outlier_rate` scaled by `outlier_scale`, RNE to BF16) with torch's
+    generator seeded 2000 + 3*layer + j, so the values differ from
+    `stack_layer`'s.  Used where 96 full matrices must be made quickly (the
+    timed stack); returns three int16 tensors holding the BF16 patterns."""
+    import torch
+    sigma = float(stack_sigmas(n_layers)[layer])
+    out = []
+    for j, (rows, cols) in enumerate(((ffn, d_model), (ffn, d_model), (d_model, ffn))):
+        g = torch.Generator(device=device)
+        g.manual_seed(2000 + 3 * layer + j)
+        w = torch.randn(rows, cols, generator=g, device=device, dtype=torch.float32) * sigma
+        if outlier_rate > 0:
+            mask = torch.rand(rows, cols, generator=g, device=device) < outlier_rate
+            w = torch.where(mask, w * outlier_scale, w)
+        out.append(w.to(torch.bfloat16).view(torch.int16))
+        del w
+    return tuple(out)
 
 
 def mlp_block(d_model: int = 4096, ffn: int = 14336, sigma: float = 0.02,

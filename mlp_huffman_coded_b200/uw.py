@@ -83,6 +83,10 @@ _SIGS = {
                                             C.POINTER(C.c_int32), C.c_int32]),
     "uw_mlp_block": (C.c_int, [C.POINTER(Matrix), C.POINTER(Matrix), C.POINTER(Matrix), C.POINTER(C.c_int32),
                                _P, C.c_int32, _P, _P, C.c_size_t, _P]),
+    "uw_mlp_stack_workspace_bytes": (C.c_size_t, [C.POINTER(C.POINTER(Matrix)), C.POINTER(C.c_int32), C.c_int32,
+                                                  C.c_int32]),
+    "uw_mlp_stack": (C.c_int, [C.POINTER(C.POINTER(Matrix)), C.POINTER(C.c_int32), C.c_int32, _P, C.c_int32, _P,
+                               _P, C.c_size_t, _P]),
     "uw_autotune": (C.c_int, [C.POINTER(Matrix), C.POINTER(C.c_int32), C.c_int32, C.c_int32, _P, _P, _P,
                               C.c_size_t, _P, C.c_size_t, C.POINTER(C.c_int32), C.POINTER(C.c_float), _P]),
     "uw_status_string": (C.c_char_p, [C.c_int]),
@@ -277,11 +281,11 @@ class DeviceMatrix:
 
     @property
     def rows(self):
-        return self.enc.rows
+        return int(self.mat.L.rows)
 
     @property
     def cols(self):
-        return self.enc.cols
+        return int(self.mat.L.cols)
 
     def prepare_direct_palette(self, ws: Workspace, stream=None, keep_idx4: bool = True):
         """Load-time preparation of the direct-palette form: transcode to 4-bit
@@ -369,6 +373,32 @@ def mlp_block(gate: DeviceMatrix, up: DeviceMatrix, down: DeviceMatrix, pipeline
               stream=None):
     _check(lib().uw_mlp_block(C.byref(gate.mat), C.byref(up.mat), C.byref(down.mat), _pipes(pipelines),
                               _ptr(x), x.shape[0], _ptr(y), ws.ptr, ws.nbytes, _stream(stream)), "uw_mlp_block")
+
+
+def _stack_args(layers, pipelines):
+    """layers: [(gate, up, down), ...] DeviceMatrix triples; pipelines: one
+    triple per layer (or one triple for every layer)."""
+    mats = [m for triple in layers for m in triple]
+    if len(pipelines) == 3 and not hasattr(pipelines[0], "__len__"):
+        pipelines = [pipelines] * len(layers)
+    pipes = [int(p) for triple in pipelines for p in triple]
+    if len(mats) != 3 * len(layers) or len(pipes) != len(mats):
+        raise ValueError("one (gate, up, down) triple and one pipeline triple per layer")
+    arr = (C.POINTER(Matrix) * len(mats))(*[C.pointer(m.mat) for m in mats])
+    return arr, (C.c_int32 * len(pipes))(*pipes), len(layers)
+
+
+def mlp_stack_workspace_bytes(layers, pipelines, batch: int) -> int:
+    arr, pipes, n = _stack_args(layers, pipelines)
+    return int(lib().uw_mlp_stack_workspace_bytes(arr, pipes, n, batch))
+
+
+def mlp_stack(layers, pipelines, x, y, ws: Workspace, stream=None):
+    """One decode step's MLP work through the stack: y = MLP_{L-1}(...
+    MLP_0(x)) (uw_mlp_stack)."""
+    arr, pipes, n = _stack_args(layers, pipelines)
+    _check(lib().uw_mlp_stack(arr, pipes, n, _ptr(x), x.shape[0], _ptr(y), ws.ptr, ws.nbytes, _stream(stream)),
+           "uw_mlp_stack")
 
 
 def autotune(dm: DeviceMatrix, batches, reps: int, x, y, ws: Workspace, flush=None, stream=None):

@@ -208,3 +208,22 @@ def test_pack_offsets_pointing_outside_the_pack_are_reported_not_faulted():
     ws.check("after restoring the offsets")
     ok, err, rms = within_tol(to_host_u16(y), *gemm_ref(w, x_host))
     assert ok, (err, rms)
+
+
+def test_workspace_shared_by_matrices_with_different_tile_counts():
+    """One workspace serves GEMMs whose plans differ (96 and 8 row tiles,
+    every tile split over several CTAs): each call leaves nothing that
+    changes the next one, so outputs equal those of fresh workspaces."""
+    big = device_matrix(synth.weight_matrix(12288, 4096, 0.02, 1e-4, 100.0, 95))
+    small = device_matrix(synth.weight_matrix(1024, 4096, 0.02, 1e-4, 100.0, 96))
+    x = to_dev(synth.activations(8, 4096, 97))
+
+    def run(dm, ws):
+        y = empty_bf16(8, int(dm.mat.L.rows))
+        uw.gemm_direct_palette(dm, x, y, ws)
+        ws.check()
+        return to_host_u16(y)
+    fresh = {id(dm): run(dm, uw.Workspace(uw.workspace_bytes(dm, uw.PIPE_DIRECT, 8))) for dm in (big, small)}
+    shared = uw.Workspace(max(uw.workspace_bytes(dm, uw.PIPE_DIRECT, 8) for dm in (big, small)))
+    for dm in (big, small, big, small, big):
+        assert np.array_equal(run(dm, shared), fresh[id(dm)])

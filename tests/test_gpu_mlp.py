@@ -118,3 +118,86 @@ def test_autotune_picks_the_fastest_it_measured():
     dm.mat.pack = None
     choice, us = uw.autotune(dm, [4], 3, x, y, ws)
     assert np.isinf(us[0, 3]) and choice[0] != 3
+
+
+def _chained_blocks(layers, dms, pipes, x):
+    """Layer outputs of uw_mlp_block calls chained through the host, each
+    checked against the float64 oracle given that layer's own input."""
+    B = x.shape[0]
+    h, outs = x, []
+    for (g, u, dn), dl, p in zip(layers, dms, pipes):
+        ws = uw.Workspace(uw.mlp_workspace_bytes(*dl, p, B))
+        y = empty_bf16(B, g.shape[1])
+        uw.mlp_block(*dl, p, to_dev(h), y, ws)
+        ws.check("block")
+        h_next = to_host_u16(y)
+        ok, err, rms = mlp_check(h_next, g, u, dn, h)
+        assert ok, (len(outs), p, err, rms)
+        outs.append(h_next)
+        h = h_next
+    return outs
+
+
+@pytest.mark.parametrize("B", [1, 8, 33])
+def test_stack_equals_chained_blocks(B):
+    """Three layers (d = 512; ffn 1536, 1024, 1536; a different pipeline mix
+    per layer): uw_mlp_stack equals the blocks chained on the host bit for
+    bit, and each layer meets the MLP bar against the oracle."""
+    d = 512
+    layers = [_block(d, ffn, seed) for ffn, seed in ((1536, 71), (1024, 74), (1536, 77))]
+    dms = [[device_matrix(m) for m in triple] for triple in layers]
+    pipes = [[3, 3, 3], [1, 3, 2], [3, 0, 3]]
+    x = synth.activations(B, d, 80)
+    outs = _chained_blocks(layers, dms, pipes, x)
+    ws = uw.Workspace(uw.mlp_stack_workspace_bytes(dms, pipes, B))
+    y = empty_bf16(B, d)
+    uw.mlp_stack(dms, pipes, to_dev(x), y, ws)
+    ws.check("stack")
+    assert np.array_equal(to_host_u16(y), outs[-1])
+    # a one-layer stack is the block itself
+    ws1 = uw.Workspace(uw.mlp_stack_workspace_bytes(dms[:1], pipes[:1], B))
+    y1 = empty_bf16(B, d)
+    uw.mlp_stack(dms[:1], pipes[:1], to_dev(x), y1, ws1)
+    ws1.check("stack")
+    assert np.array_equal(to_host_u16(y1), outs[0])
+
+
+def test_stack_rejects_bad_arguments():
+    d = 256
+    a = [device_matrix(m) for m in _block(d, 512, 81)]
+    b = [device_matrix(m) for m in _block(2 * d, 512, 84)]  # maps 512 -> 512: does not chain with a
+    x = to_dev(synth.activations(2, d, 85))
+    y = empty_bf16(2, d)
+    assert uw.mlp_stack_workspace_bytes([a, b], [3, 3, 3], 2) == 0
+    need = uw.mlp_stack_workspace_bytes([a, a], [3, 3, 3], 2)
+    assert need > uw.mlp_workspace_bytes(*a, [3, 3, 3], 2)
+    small = uw.Workspace(need - 256)
+    with pytest.raises(uw.UwError) as e:
+        uw.mlp_stack([a, a], [3, 3, 3], x, y, small)
+    assert e.value.status == uw.UW_ERR_WORKSPACE_TOO_SMALL
+    ws = uw.Workspace(need)
+    with pytest.raises(uw.UwError) as e:
+        uw.mlp_stack([a, b], [3, 3, 3], x, y, ws)
+    assert e.value.status == uw.UW_ERR_INVALID_ARG
+
+
+@pytest.fixture(scope="module")
+def two_full_layers():
+    layers = [synth.stack_layer(layer) for layer in (0, 1)]
+    return layers, [[device_matrix(m) for m in triple] for triple in layers]
+
+
+@pytest.mark.parametrize("B", [1, 64])
+def test_full_size_two_layer_stack(two_full_layers, B):
+    """The first two layers of the 32-layer stack (gate/up 14336x4096, down
+    4096x14336, 1e-3 outliers), direct palette throughout, in the launch
+    configuration the stack benchmark times."""
+    layers, dms = two_full_layers
+    pipes = [[3, 3, 3]] * 2
+    x = synth.activations(B, 4096, 86)
+    outs = _chained_blocks(layers, dms, pipes, x)
+    ws = uw.Workspace(uw.mlp_stack_workspace_bytes(dms, pipes, B))
+    y = empty_bf16(B, 4096)
+    uw.mlp_stack(dms, pipes, to_dev(x), y, ws)
+    ws.check("stack")
+    assert np.array_equal(to_host_u16(y), outs[-1])

@@ -57,7 +57,7 @@ def _scratch_need(rows, B, sms):
     n_ntiles = -(-B // 256)
     ntile = -(-(-(-B // n_ntiles)) // 16) * 16
     tiles = -(-rows // 128) * n_ntiles
-    counters = -(-tiles * 4 // 256) * 256
+    counters = 64 * 1024  # fixed region, the same for every plan
     return 256 + counters + (tiles + sms) * ntile * 128 * 4
 
 
