@@ -301,6 +301,18 @@ UW_API uw_status uw_decode_full(const uw_matrix* m, uint16_t* out_bf16, void* wo
 UW_API uw_status uw_decode_exponent_only(const uw_matrix* m, uint8_t* out_exp8, void* workspace,
                                   size_t workspace_bytes, void* stream);
 
+/* Full decode of selected rows (an embedding lookup on a compressed
+ * embedding table; section "How to compress model weights effectively"
+ * names embeddings among the matrices the page leaves raw): out_bf16
+ * [n_rows, cols] (device) row i = row rows[i] of W, bit for bit.  rows:
+ * device int32[n_rows]; repeats allowed.  Only the chunks that hold a
+ * requested row are decoded.  Errors as uw_decode_full, plus
+ * UW_ERR_INVALID_ARG for n_rows < 0 or NULL rows; a row id outside
+ * [0, rows) is found on the device: that output row is zeros and the
+ * status word records UW_ERR_INVALID_ARG. */
+UW_API uw_status uw_decode_rows(const uw_matrix* m, const int32_t* rows, int32_t n_rows, uint16_t* out_bf16,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* Palette transcode (section "Four ways to use compressed weights"):
  * out_idx4[rows*cols/2] (device) = 4-bit palette index per element in the
  * idx4 layout, 0 in verbatim groups; a quarter of the full decode's write

@@ -1,5 +1,6 @@
 // Chunked-bitstream Huffman decoders: full BF16 decode, exponent-only
-// decode and 4-bit palette transcode.
+// decode, 4-bit palette transcode, and the full decode of selected rows
+// (an embedding lookup).
 //
 // Method: Cloudflare, "Unweight: how we compressed an LLM 22% without
 // sacrificing quality", section "Four ways to use compressed weights" (the
@@ -7,19 +8,28 @@
 // element) and section "How to compress model weights effectively" (palette,
 // Huffman-coded exponent, verbatim 64-element rows).
 //
-// Parallel structure: the stream is cut into chunks of `chunk_groups`
-// 64-element groups, each with its own start bit, so one thread decodes one
-// chunk from start to end.  The canonical code is decoded through a table in
-// shared memory indexed by the next 11 bits, which yields every whole code in
-// them at once (up to 4 symbols: their outputs and cumulative lengths);
-// longer codes (rare: the tail of the exponent distribution) fall back to the
-// canonical first-code comparison.  Each 16-symbol quarter of a group is
-// gathered in 64-bit registers and goes to global memory in one store;
-// sign+mantissa bytes are fetched with a 16-byte load issued before the
-// quarter is decoded.
-// Verbatim groups (flag bit set) are copied from the verbatim store instead
-// and consume no stream bits.
+// Work split.  The stream is cut into chunks of `chunk_groups` 64-element
+// groups, each with its own start bit.  A warp takes 32 consecutive chunks
+// (one per lane) in two steps:
+//   1. each lane decodes its chunk's coded groups into 4-bit palette indices:
+//      a 32-bit window over three prefetched stream words (funnel shift), one
+//      shared-memory table lookup per 11 bits yielding every whole code in
+//      them (up to 4 indices, their total length and count), and the indices
+//      packed 8 to a word into the warp's shared-memory stage.  Codes longer
+//      than the table (the rare tail of the exponent distribution) take the
+//      canonical first-code comparison.  This step is the same whatever the
+//      output format;
+//   2. the warp writes the 32 chunks' groups together: consecutive lanes take
+//      consecutive 16-byte pieces of the output, so every store (and, for the
+//      full decode, every sign+mantissa load) is coalesced.  Indices become
+//      exponent bytes by a byte-permute palette lookup; verbatim groups come
+//      from the verbatim store.
+// A chunk whose codes do not end exactly at the next chunk's offset, or an
+// invalid code, records UW_ERR_CORRUPT; every stream read stays inside the
+// stream and every verbatim read inside the store.
 #include <cuda_runtime.h>
+
+#include <algorithm>
 
 #include "uw_device.cuh"
 #include "uw_internal.h"
@@ -30,7 +40,7 @@ namespace {
 
 constexpr int kLutBits = 11;
 constexpr int kLutSize = 1 << kLutBits;
-constexpr int kDecodeThreads = 256;
+constexpr int kStageBudget = 48 * 1024;  // per block: index stage + group info
 
 enum DecodeMode { kFull = 0, kExp8 = 1, kIdx4 = 2 };
 
@@ -41,36 +51,40 @@ struct DecodeParams {
   const uint32_t* vflags;
   const uint32_t* vprefix;
   const uint16_t* verbatim;
+  const int32_t* rows;  // row gather: the rows to decode (device), else NULL
   void* out;
   uint32_t* status;
   int64_t n_groups;
   int64_t n_verbatim;
   int64_t n_chunks;
   int64_t stream_words;
+  int64_t n_rows;           // rows of the matrix
+  int64_t n_items;          // warp work items: 32-chunk batches (of each gathered row)
+  int32_t batches_per_row;  // row gather
   int32_t chunk_groups;
   int32_t gpr;  // groups per row
   int32_t wpr;  // flag words per row
   int32_t max_len;
-  uint8_t palette[16];
+  int32_t mixed;  // the palette lookup needs the top-bit tables
+  PaletteTables pal;
   uint8_t code_len[16];
 };
 
 struct DecodeTables {
-  uint16_t lut[kLutSize];  // sym | len << 4 | exp << 8; len 0 = not in table
-  // Several symbols per lookup: for each 11-bit prefix, the whole codes it
-  // holds (at most 4): bits 0..31 their outputs (exponent bytes, or palette
-  // nibbles for the transcode), bits 32..47 the cumulative code lengths
-  // after 1..4 symbols (4 bits each), bits 48..50 the count (0: the first
-  // code is longer than the table).
-  uint64_t multi[kLutSize];
-  uint32_t first[17];      // first canonical code of each length
-  uint32_t count[17];      // codes of each length
-  uint32_t offset[17];     // index of the first symbol of each length
-  uint8_t sorted[16];      // symbols in (length, index) order
-  uint8_t palette[16];
+  // Every whole code inside each 11-bit prefix (at most 4): x = their
+  // palette indices (4 bits each, first code lowest) | cumulative lengths
+  // after 1..4 codes (4 bits each) << 16; y = count | total length << 8
+  // (count 0: the first code is longer than the table).
+  uint2 multi[kLutSize];
+  uint32_t first[17];   // first canonical code of each length
+  uint32_t count[17];   // codes of each length
+  uint32_t offset[17];  // index of the first symbol of each length
+  uint8_t sorted[16];   // symbols in (length, index) order
 };
 
-__device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables& t, bool mode_idx4) {
+// lut: kLutSize words of scratch (the first code of each prefix, sym |
+// len << 4, len 0 = longer than the table), needed only while building.
+__device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables& t, uint16_t* lut) {
   if (threadIdx.x == 0) {
     for (int l = 0; l <= 16; ++l) t.count[l] = 0;
     for (int i = 0; i < 16; ++i)
@@ -86,7 +100,6 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables
     for (int l = 1; l <= 15; ++l)
       for (int i = 0; i < 16; ++i)
         if (p.code_len[i] == l) t.sorted[k++] = static_cast<uint8_t>(i);
-    for (int i = 0; i < 16; ++i) t.palette[i] = p.palette[i];
   }
   __syncthreads();
   const int lim = p.max_len < kLutBits ? p.max_len : kLutBits;
@@ -96,200 +109,297 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables
       const uint32_t code = static_cast<uint32_t>(v) >> (kLutBits - l);
       const uint32_t d = code - t.first[l];
       if (t.count[l] && d < t.count[l]) {
-        const int sym = t.sorted[t.offset[l] + d];
-        ent = static_cast<uint16_t>(sym | (l << 4) | (p.palette[sym] << 8));
+        ent = static_cast<uint16_t>(t.sorted[t.offset[l] + d] | (l << 4));
         break;
       }
     }
-    t.lut[v] = ent;
+    lut[v] = ent;
   }
   __syncthreads();
-  // chain single-symbol lookups inside the 11-bit prefix: a code shorter than
+  // chain single-code lookups inside the 11-bit prefix: a code shorter than
   // the bits left is decoded correctly whatever the zero padding (prefix-free)
   for (int v = threadIdx.x; v < kLutSize; v += blockDim.x) {
-    uint64_t payload = 0, cum = 0;
+    uint32_t idx = 0, cum = 0;
     int used = 0, n = 0;
     while (n < 4 && used < kLutBits) {
-      const uint32_t e = t.lut[(static_cast<uint32_t>(v) << used) & (kLutSize - 1)];
+      const uint32_t e = lut[(static_cast<uint32_t>(v) << used) & (kLutSize - 1)];
       const int l = (e >> 4) & 15;
       if (l == 0 || l > kLutBits - used) break;
-      const uint64_t out = mode_idx4 ? (e & 15u) : (e >> 8);
-      payload |= out << (mode_idx4 ? 4 * n : 8 * n);
+      idx |= (e & 15u) << (4 * n);
       used += l;
-      cum |= static_cast<uint64_t>(used) << (4 * n);
+      cum |= static_cast<uint32_t>(used) << (4 * n);
       ++n;
     }
-    t.multi[v] = payload | (cum << 32) | (static_cast<uint64_t>(n) << 48);
+    t.multi[v] = make_uint2(idx | (cum << 16), static_cast<uint32_t>(n) | (static_cast<uint32_t>(used) << 8));
   }
   __syncthreads();
 }
 
-// A code longer than the table (rare: the tail of the exponent distribution)
-// by canonical first-code comparison, as a single-symbol entry (sym | len << 4
-// | exponent << 8).  On an invalid code records UW_ERR_CORRUPT and returns a
-// length-1 entry so decoding stays bounded.
-__device__ __forceinline__ uint32_t decode_long(const DecodeTables& t, int max_len, uint32_t* status,
-                                             uint64_t win) {
+// A code longer than the table by canonical first-code comparison over the
+// left-aligned 32-bit window: symbol | length << 4.  An invalid code records
+// UW_ERR_CORRUPT and reads as symbol 0 of length 1, so decoding stays bounded.
+__device__ __noinline__ uint32_t decode_long(const DecodeTables& t, int max_len, uint32_t* status, uint32_t win) {
   for (int l = kLutBits + 1; l <= max_len; ++l) {
-    const uint32_t code = static_cast<uint32_t>(win >> (64 - l));
-    const uint32_t d = code - t.first[l];
-    if (t.count[l] && d < t.count[l]) {
-      const int sym = t.sorted[t.offset[l] + d];
-      return static_cast<uint32_t>(sym | (l << 4) | (t.palette[sym] << 8));
-    }
+    const uint32_t d = (win >> (32 - l)) - t.first[l];
+    if (t.count[l] && d < t.count[l]) return t.sorted[t.offset[l] + d] | (static_cast<uint32_t>(l) << 4);
   }
   record_status(status, UW_ERR_CORRUPT);
   return 1u << 4;
 }
 
-template <int MODE>
-__global__ void __launch_bounds__(kDecodeThreads, 7) decode_kernel(const DecodeParams p) {
-  __shared__ DecodeTables t;
-  build_tables(p, t, MODE == kIdx4);
-  const int64_t last_word = p.stream_words - 1;
-  for (int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; c < p.n_chunks;
-       c += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const uint32_t b0 = p.off[c];
-    const uint32_t b1 = p.off[c + 1];
-    // left-aligned bit window over the stream
-    int64_t wi = b0 >> 5;
-    const uint32_t sh = b0 & 31;
-    uint64_t win = (static_cast<uint64_t>(__ldg(p.stream + min(wi, last_word))) << 32) |
-                   __ldg(p.stream + min(wi + 1, last_word));
-    win <<= sh;
-    int nb = 64 - static_cast<int>(sh);
-    wi += 2;
-    uint32_t consumed = 0;
+// Word w of a lane's stage region (8 words per chunk group): 4-word units
+// XOR-swizzled by the lane so lanes writing the same word mostly hit
+// different banks; a unit stays contiguous (16-byte reads).  umask + 1 is a
+// power of two dividing the region's unit count, so the swizzle stays inside
+// the region.
+__device__ __forceinline__ uint32_t stage_word(int lane, int w, int cg, int umask) {
+  return static_cast<uint32_t>(lane * 8 * cg + (((w >> 2) ^ (lane & umask)) << 2) + (w & 3));
+}
 
-    const int64_t g0 = c * p.chunk_groups;
-    const int64_t g1 = min(g0 + p.chunk_groups, p.n_groups);
-    for (int64_t g = g0; g < g1; ++g) {
-      const int64_t r = g / p.gpr;
-      const int32_t j = static_cast<int32_t>(g - r * p.gpr);
+// Step 1: the lane decodes chunk c into its stage region (coded groups at
+// their slots, 8 words each) and records every group's source in info[]:
+// -1 coded, >= 0 verbatim slot, -2 unreadable verbatim slot (written as
+// zeros), -3 past the matrix.
+__device__ __forceinline__ void decode_chunk(const DecodeParams& p, const DecodeTables& t, int64_t c, int lane,
+                                             uint32_t* stage, int32_t* info, int umask) {
+  const int cg = p.chunk_groups;
+  const int64_t g0 = c * cg;
+  const int64_t g1 = min(g0 + cg, p.n_groups);
+  int64_t r = g0 / p.gpr;
+  int32_t j = static_cast<int32_t>(g0 - r * p.gpr);
+  uint32_t coded = 0;
+  for (int s = 0; s < cg; ++s) {
+    int32_t v = -3;
+    if (g0 + s < g1) {
       const int64_t fw = r * p.wpr + (j >> 5);
-      const uint32_t flags = __ldg(p.vflags + fw);
+      const uint32_t fl = __ldg(p.vflags + fw);
       const uint32_t bit = 1u << (j & 31);
-      const int64_t e0 = g * 64;
-      if (flags & bit) {
-        // verbatim group: raw words from the store, no stream bits
-        int64_t slot = __ldg(p.vprefix + fw) + __popc(flags & (bit - 1));
-        if (slot >= p.n_verbatim) {
-          // corrupt flags or prefixes: report, and read nothing outside the
-          // store (slot 0 stands in; a store-less matrix writes zeros)
+      if (fl & bit) {
+        const int64_t slot = static_cast<int64_t>(__ldg(p.vprefix + fw)) + __popc(fl & (bit - 1));
+        if (slot < p.n_verbatim) {
+          v = static_cast<int32_t>(slot);
+        } else {
           record_status(p.status, UW_ERR_CORRUPT);
-          slot = 0;
+          v = -2;
         }
-        const bool have = p.n_verbatim > 0;
-        const uint4 zero = make_uint4(0, 0, 0, 0);
-        const uint4* src = reinterpret_cast<const uint4*>(p.verbatim + slot * 64);
-        if (MODE == kFull) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + e0);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) dst[k] = have ? __ldg(src + k) : zero;
-        } else if (MODE == kExp8) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + e0);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint4 a = have ? __ldg(src + 2 * k) : zero, b = have ? __ldg(src + 2 * k + 1) : zero;
-            // exponent = bits 7..14 of each 16-bit word: take the byte that
-            // straddles them after a 7-bit right shift of each word pair
-            const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-            uint32_t o[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint32_t lo = (w[2 * q] >> 7) & 0x00FF00FFu;
-              const uint32_t hi = (w[2 * q + 1] >> 7) & 0x00FF00FFu;
-              o[q] = __byte_perm(lo, hi, 0x6420);
-            }
-            dst[k] = make_uint4(o[0], o[1], o[2], o[3]);
-          }
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + e0 / 2);
-          dst[0] = make_uint4(0, 0, 0, 0);
-          dst[1] = make_uint4(0, 0, 0, 0);
-        }
-        continue;
+      } else {
+        v = -1;
+        coded |= 1u << s;
       }
-      // quarters of 16 symbols, not unrolled (code size: the instruction
-      // cache, not arithmetic, limited the fully unrolled group)
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        // sign+mantissa bytes of this quarter: issued before its 16 symbols
-        uint4 smq = make_uint4(0, 0, 0, 0);
-        if (MODE == kFull) smq = __ldg(reinterpret_cast<const uint4*>(p.sm + e0) + q);
-        // 16 symbols -> 16 exponent bytes (a0 | a1 << 64) or 16 nibbles (a0),
-        // several symbols per table lookup
-        uint64_t a0 = 0, a1 = 0;
-        int pos = 0;
-        while (pos < 16) {
-          if (nb < 32) {
-            win |= static_cast<uint64_t>(__ldg(p.stream + min(wi, last_word))) << (32 - nb);
-            ++wi;
-            nb += 32;
-          }
-          const uint64_t ent = t.multi[static_cast<uint32_t>(win >> (64 - kLutBits))];
-          const int cnt = static_cast<int>((ent >> 48) & 7);
-          int k, len;
-          uint64_t pay;
-          if (cnt == 0) {  // a code longer than the table
-            const uint32_t e = decode_long(t, p.max_len, p.status, win);
-            k = 1;
-            len = static_cast<int>((e >> 4) & 15);
-            pay = MODE == kIdx4 ? (e & 15u) : (e >> 8);
-          } else {
-            k = min(cnt, 16 - pos);
-            len = static_cast<int>((ent >> (32 + 4 * (k - 1))) & 15);
-            pay = ent & ((MODE == kIdx4 ? (1ull << (4 * k)) : (1ull << (8 * k))) - 1);
-          }
-          if (MODE == kIdx4) {
-            a0 |= pay << (4 * pos);
-          } else {
-            const int bp = 8 * pos;
-            if (pos < 8) {
-              a0 |= pay << bp;
-              if (pos + k > 8) a1 |= pay >> (64 - bp);
-            } else {
-              a1 |= pay << (bp - 64);
-            }
-          }
-          win <<= len;
-          nb -= len;
-          consumed += static_cast<uint32_t>(len);
-          pos += k;
-        }
-        const uint32_t v[4] = {static_cast<uint32_t>(a0), static_cast<uint32_t>(a0 >> 32), static_cast<uint32_t>(a1),
-                               static_cast<uint32_t>(a1 >> 32)};
-        if (MODE == kFull) {
-          const uint4 s = smq;
-          uint32_t o[8];
-          rebuild4(s.x, v[0], o[0], o[1]);
-          rebuild4(s.y, v[1], o[2], o[3]);
-          rebuild4(s.z, v[2], o[4], o[5]);
-          rebuild4(s.w, v[3], o[6], o[7]);
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + e0 + 16 * q);
-          dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-          dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
-        } else if (MODE == kExp8) {
-          *reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + e0 + 16 * q) =
-              make_uint4(v[0], v[1], v[2], v[3]);
-        } else {
-          *reinterpret_cast<uint2*>(static_cast<uint8_t*>(p.out) + e0 / 2 + 8 * q) = make_uint2(v[0], v[1]);
-        }
+      if (++j == p.gpr) {
+        j = 0;
+        ++r;
       }
     }
-    if (consumed != b1 - b0) record_status(p.status, UW_ERR_CORRUPT);
+    info[lane * cg + s] = v;
+  }
+  const uint32_t b0 = __ldg(p.off + c), b1 = __ldg(p.off + c + 1);
+  const int64_t last_word = p.stream_words - 1;
+  int64_t wi = b0 >> 5;
+  uint32_t w0 = __ldg(p.stream + min(wi, last_word));
+  uint32_t w1 = __ldg(p.stream + min(wi + 1, last_word));
+  uint32_t w2 = __ldg(p.stream + min(wi + 2, last_word));
+  wi += 3;
+  int bp = static_cast<int>(b0 & 31);
+  uint32_t consumed = 0;
+  const int total = 64 * __popc(coded);
+  int done = 0;
+  uint32_t acc_lo = 0, acc_hi = 0;  // pending indices, first lowest
+  int nacc = 0;                     // indices pending (< 8 between steps)
+  uint32_t left = coded;            // coded groups not started yet
+  int slot = 0, wq = 8;             // current group's slot, words written into it
+  // Both steps are written to compile to selects and predicated memory
+  // operations rather than branches: lanes of a warp flush and refill at
+  // different times.
+  auto push = [&](uint32_t idx, int cnt) {
+    const int sh = 4 * nacc;
+    const uint64_t a = (static_cast<uint64_t>(acc_hi) << 32 | acc_lo) | (static_cast<uint64_t>(idx) << sh);
+    nacc += cnt;
+    const bool full = nacc >= 8;  // 8 indices -> the stage
+    const bool start = full && wq == 8;
+    slot = start ? __ffs(left) - 1 : slot;
+    left = start ? left & (left - 1) : left;
+    wq = start ? 0 : wq;
+    if (full) stage[stage_word(lane, slot * 8 + wq, cg, umask)] = static_cast<uint32_t>(a);
+    wq += full ? 1 : 0;
+    acc_lo = full ? static_cast<uint32_t>(a >> 32) : static_cast<uint32_t>(a);
+    acc_hi = full ? 0u : static_cast<uint32_t>(a >> 32);
+    nacc -= full ? 8 : 0;
+  };
+  auto advance = [&](int len) {
+    bp += len;
+    consumed += static_cast<uint32_t>(len);
+    const bool cross = bp >= 32;
+    uint32_t nw = 0;
+    if (cross) nw = __ldg(p.stream + min(wi, last_word));
+    bp -= cross ? 32 : 0;
+    w0 = cross ? w1 : w0;
+    w1 = cross ? w2 : w1;
+    w2 = cross ? nw : w2;
+    wi += cross ? 1 : 0;
+  };
+  // whole lookups while at least 4 indices remain (two per check)
+  auto step = [&]() {
+    const uint32_t win = __funnelshift_l(w1, w0, bp);
+    const uint2 e = t.multi[win >> (32 - kLutBits)];
+    int cnt = static_cast<int>(e.y & 7);
+    uint32_t idx = e.x & 0xFFFFu;
+    int len = static_cast<int>(e.y >> 8);
+    if (cnt == 0) {
+      const uint32_t d = decode_long(t, p.max_len, p.status, win);
+      idx = d & 15u;
+      len = static_cast<int>(d >> 4);
+      cnt = 1;
+    }
+    push(idx, cnt);
+    advance(len);
+    done += cnt;
+  };
+  while (total - done >= 8) {
+    step();
+    step();
+  }
+  while (total - done >= 4) step();
+  // the last indices one code at a time
+  while (done < total) {
+    const uint32_t win = __funnelshift_l(w1, w0, bp);
+    const uint2 e = t.multi[win >> (32 - kLutBits)];
+    uint32_t idx;
+    int len;
+    if ((e.y & 7) == 0) {
+      const uint32_t d = decode_long(t, p.max_len, p.status, win);
+      idx = d & 15u;
+      len = static_cast<int>(d >> 4);
+    } else {
+      idx = e.x & 15u;
+      len = static_cast<int>((e.x >> 16) & 15);
+    }
+    push(idx, 1);
+    advance(len);
+    ++done;
+  }
+  if (consumed != b1 - b0) record_status(p.status, UW_ERR_CORRUPT);
+}
+
+__device__ __forceinline__ uint32_t lookup4(const DecodeParams& p, uint32_t nib) {
+  return p.mixed ? lookup4_mixed(p.pal, nib) : lookup4_uniform(p.pal, nib);
+}
+
+// Exponent bytes of 16 BF16 words given as two uint4 (elements in order).
+__device__ __forceinline__ uint4 exponents16(const uint4& a, const uint4& b) {
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t o[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    // exponent = bits 7..14 of each 16-bit word: after a 7-bit right shift
+    // each word's exponent is its low byte
+    const uint32_t lo = (w[2 * q] >> 7) & 0x00FF00FFu;
+    const uint32_t hi = (w[2 * q + 1] >> 7) & 0x00FF00FFu;
+    o[q] = __byte_perm(lo, hi, 0x6420);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// Step 2: the output pieces of batch groups [gl0, gl1) (batch group gi is
+// slot gi % cg of lane gi / cg's chunk; matrix group g_batch0 + gi); og0 is
+// the output group of batch group gl0.  `zero`: write zeros.
+template <int MODE>
+__device__ __forceinline__ void emit_groups(const DecodeParams& p, const uint32_t* stage, const int32_t* info,
+                                            int umask, int64_t g_batch0, int gl0, int gl1, int64_t og0,
+                                            bool zero) {
+  constexpr int kPieces = MODE == kIdx4 ? 2 : (MODE == kExp8 ? 4 : 8);  // 16-byte pieces per group
+  const int cg = p.chunk_groups;
+  const int lane = threadIdx.x & 31;
+  const int n = (gl1 - gl0) * kPieces;
+  for (int pc = lane; pc < n; pc += 32) {
+    const int gi = gl0 + pc / kPieces;
+    const int q = pc % kPieces;
+    const int L = gi / cg, s = gi - L * cg;
+    const int32_t v = zero ? -2 : info[gi];
+    const int64_t og = og0 + (gi - gl0);
+    uint4 o = make_uint4(0, 0, 0, 0);
+    if (MODE == kIdx4) {
+      if (v == -1) o = *reinterpret_cast<const uint4*>(stage + stage_word(L, s * 8 + 4 * q, cg, umask));
+      reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + og * 32)[q] = o;
+    } else if (MODE == kExp8) {
+      if (v == -1) {
+        const uint2 nw = *reinterpret_cast<const uint2*>(stage + stage_word(L, s * 8 + 2 * q, cg, umask));
+        o = make_uint4(lookup4(p, nw.x), lookup4(p, nw.x >> 16), lookup4(p, nw.y), lookup4(p, nw.y >> 16));
+      } else if (v >= 0) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.verbatim + static_cast<int64_t>(v) * 64) + 2 * q;
+        o = exponents16(__ldg(src), __ldg(src + 1));
+      }
+      reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + og * 64)[q] = o;
+    } else {
+      if (v == -1) {
+        const uint32_t nw = stage[stage_word(L, s * 8 + q, cg, umask)];
+        const uint2 smv = __ldg(reinterpret_cast<const uint2*>(p.sm + (g_batch0 + gi) * 64) + q);
+        rebuild4(smv.x, lookup4(p, nw), o.x, o.y);
+        rebuild4(smv.y, lookup4(p, nw >> 16), o.z, o.w);
+      } else if (v >= 0) {
+        o = __ldg(reinterpret_cast<const uint4*>(p.verbatim + static_cast<int64_t>(v) * 64) + q);
+      }
+      reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + og * 64)[q] = o;
+    }
   }
 }
 
-}  // namespace
+template <int MODE, bool ROWS>
+__global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
+  __shared__ DecodeTables t;
+  extern __shared__ __align__(16) uint32_t dsm[];
+  build_tables(p, t, reinterpret_cast<uint16_t*>(dsm));  // the stage holds the build scratch
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int W = blockDim.x >> 5;
+  const int cg = p.chunk_groups;
+  uint32_t* stage = dsm + warp * (256 * cg);
+  int32_t* info = reinterpret_cast<int32_t*>(dsm + W * 256 * cg) + warp * 32 * cg;
+  const int units = 2 * cg;
+  const int umask = min(units & -units, 8) - 1;
+  for (int64_t it = static_cast<int64_t>(blockIdx.x) * W + warp; it < p.n_items;
+       it += static_cast<int64_t>(gridDim.x) * W) {
+    int64_t c_first, c_end, g_lo, g_hi, og0;
+    bool zero = false;
+    if (!ROWS) {
+      c_first = it * 32;
+      c_end = min(c_first + 32, p.n_chunks);
+      g_lo = c_first * cg;
+      g_hi = min(c_end * cg, p.n_groups);
+      og0 = g_lo;
+    } else {
+      const int64_t i = it / p.batches_per_row;
+      const int b = static_cast<int>(it - i * p.batches_per_row);
+      int64_t r = __ldg(p.rows + i);
+      if (r < 0 || r >= p.n_rows) {
+        // a row outside the matrix: zeros, and the status word says so
+        if (lane == 0 && b == 0) record_status(p.status, UW_ERR_INVALID_ARG);
+        zero = true;
+        r = 0;
+      }
+      const int64_t rg0 = r * p.gpr, rg1 = rg0 + p.gpr;
+      const int64_t cr0 = rg0 / cg, cr1 = (rg1 - 1) / cg + 1;
+      c_first = cr0 + static_cast<int64_t>(b) * 32;
+      c_end = min(c_first + 32, cr1);
+      if (c_first >= c_end) continue;
+      g_lo = max(c_first * cg, rg0);
+      g_hi = min(c_end * cg, rg1);
+      og0 = i * p.gpr + (g_lo - rg0);
+    }
+    const int64_t c = c_first + lane;
+    if (c < c_end && !zero) decode_chunk(p, t, c, lane, stage, info, umask);
+    __syncwarp();
+    emit_groups<MODE>(p, stage, info, umask, c_first * cg, static_cast<int>(g_lo - c_first * cg),
+                      static_cast<int>(g_hi - c_first * cg), og0, zero);
+    __syncwarp();
+  }
+}
 
-uw_status launch_decode(const uw_matrix* m, int mode, void* out, uint32_t* status, cudaStream_t s) {
+uw_status fill_params(const uw_matrix* m, void* out, uint32_t* status, DecodeParams* pp) {
   uw_status st = check_matrix(m);
   if (st != UW_OK) return st;
   if (!out || !aligned16(out)) return UW_ERR_INVALID_ARG;
-  DeviceInfo dev;
-  if ((st = device_info(&dev)) != UW_OK) return st;
-  DecodeParams p;
+  DecodeParams& p = *pp;
+  p = DecodeParams{};
   p.sm = m->sm;
   p.stream = m->stream;
   p.off = m->chunk_bit_off;
@@ -302,25 +412,75 @@ uw_status launch_decode(const uw_matrix* m, int mode, void* out, uint32_t* statu
   p.n_verbatim = m->L.n_verbatim;
   p.n_chunks = m->L.n_chunks;
   p.stream_words = m->L.stream_words;
+  p.n_rows = m->L.rows;
   p.chunk_groups = m->L.chunk_groups;
   p.gpr = static_cast<int32_t>(m->L.cols / 64);
   p.wpr = m->L.words_per_row;
   p.max_len = m->cb.max_len;
-  for (int i = 0; i < 16; ++i) {
-    p.palette[i] = m->cb.palette[i];
-    p.code_len[i] = m->cb.code_len[i];
-  }
-  const int64_t blocks_needed = (p.n_chunks + kDecodeThreads - 1) / kDecodeThreads;
-  const int64_t max_blocks = static_cast<int64_t>(dev.sm_count) * 8;
-  const int grid = static_cast<int>(blocks_needed < max_blocks ? blocks_needed : max_blocks);
-  if (grid <= 0) return UW_OK;
-  switch (mode) {
-    case kFull: decode_kernel<kFull><<<grid, kDecodeThreads, 0, s>>>(p); break;
-    case kExp8: decode_kernel<kExp8><<<grid, kDecodeThreads, 0, s>>>(p); break;
-    default: decode_kernel<kIdx4><<<grid, kDecodeThreads, 0, s>>>(p); break;
-  }
+  bool mixed = false;
+  p.pal = palette_tables(m->cb.palette, m->cb.code_len, &mixed);
+  p.mixed = mixed ? 1 : 0;
+  for (int i = 0; i < 16; ++i) p.code_len[i] = m->cb.code_len[i];
+  return UW_OK;
+}
+
+// Warps per block: the index stage (1 KB per chunk group per warp) and the
+// group info (128 bytes per chunk group per warp) within kStageBudget, at
+// most 8.
+int warps_per_block(int cg) { return std::max(1, std::min(8, kStageBudget / (cg * 1152))); }
+
+template <int MODE, bool ROWS>
+uw_status launch(const DecodeParams& p, const DeviceInfo& dev, cudaStream_t s) {
+  if (p.n_items <= 0) return UW_OK;
+  const int W = warps_per_block(p.chunk_groups);
+  // (also the table build's kLutSize-word scratch)
+  const size_t smem = std::max<size_t>(static_cast<size_t>(W) * p.chunk_groups * 1152, kLutSize * 2);
+  if (cudaFuncSetAttribute(decode_kernel<MODE, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStageBudget) !=
+      cudaSuccess)
+    return UW_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<MODE, ROWS>, 32 * W, smem) !=
+      cudaSuccess)
+    return UW_ERR_CUDA;
+  const int64_t blocks_needed = (p.n_items + W - 1) / W;
+  const int64_t resident = static_cast<int64_t>(dev.sm_count) * std::max(1, per_sm);
+  const int grid = static_cast<int>(std::min(blocks_needed, resident));
+  decode_kernel<MODE, ROWS><<<grid, 32 * W, smem, s>>>(p);
   note_launch();
   return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+uw_status launch_decode(const uw_matrix* m, int mode, void* out, uint32_t* status, cudaStream_t s) {
+  DecodeParams p;
+  uw_status st = fill_params(m, out, status, &p);
+  if (st != UW_OK) return st;
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != UW_OK) return st;
+  p.n_items = (p.n_chunks + 31) / 32;
+  switch (mode) {
+    case kFull: return launch<kFull, false>(p, dev, s);
+    case kExp8: return launch<kExp8, false>(p, dev, s);
+    default: return launch<kIdx4, false>(p, dev, s);
+  }
+}
+
+uw_status launch_decode_rows(const uw_matrix* m, const int32_t* rows, int64_t n_rows, void* out, uint32_t* status,
+                             cudaStream_t s) {
+  if (n_rows < 0 || (n_rows > 0 && !rows)) return UW_ERR_INVALID_ARG;
+  DecodeParams p;
+  uw_status st = fill_params(m, out, status, &p);
+  if (st != UW_OK) return st;
+  if (n_rows == 0) return UW_OK;
+  DeviceInfo dev;
+  if ((st = device_info(&dev)) != UW_OK) return st;
+  p.rows = rows;
+  // chunks one row touches: at most gpr / cg + 2
+  const int64_t per_row = p.gpr / p.chunk_groups + 2;
+  p.batches_per_row = static_cast<int32_t>((per_row + 31) / 32);
+  p.n_items = n_rows * p.batches_per_row;
+  return launch<kFull, true>(p, dev, s);
 }
 
 }  // namespace uw

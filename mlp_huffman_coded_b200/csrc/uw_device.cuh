@@ -358,6 +358,33 @@ __device__ __forceinline__ uint32_t prmt_sx(uint32_t a, uint32_t b, uint32_t sel
   return d;
 }
 
+// Tables of a palette (host side).  *mixed: the palette entries with a code
+// (all of them when code_len is NULL) disagree in the exponent's top bit.
+inline PaletteTables palette_tables(const uint8_t* pal, const uint8_t* code_len, bool* mixed) {
+  PaletteTables t;
+  uint32_t w[4] = {0, 0, 0, 0}, b7[4] = {0, 0, 0, 0};
+  int seen0 = 0, seen1 = 0;
+  for (int i = 0; i < 16; ++i) {
+    w[i / 4] |= static_cast<uint32_t>(pal[i] | 0x80u) << (8 * (i % 4));
+    b7[i / 4] |= static_cast<uint32_t>(0xBFu | ((pal[i] >> 7) << 6)) << (8 * (i % 4));
+    if (!code_len || code_len[i]) {
+      if (pal[i] & 0x80) seen1 = 1;
+      else seen0 = 1;
+    }
+  }
+  t.lo0 = w[0];
+  t.lo1 = w[1];
+  t.hi0 = w[2];
+  t.hi1 = w[3];
+  t.b7lo0 = b7[0];
+  t.b7lo1 = b7[1];
+  t.b7hi0 = b7[2];
+  t.b7hi1 = b7[3];
+  *mixed = seen0 && seen1;
+  t.keep = seen1 ? 0xFFFFFFFFu : 0x7F7F7F7Fu;
+  return t;
+}
+
 __device__ __forceinline__ uint32_t lookup4_uniform(const PaletteTables& p, uint32_t nib) {
   const uint32_t a = prmt_sx(p.lo0, p.lo1, nib);
   const uint32_t b = prmt_sx(p.hi0, p.hi1, nib ^ 0x8888u);

@@ -1166,30 +1166,6 @@ uw_status launch_kernel(const CUtensorMap& x, const CUtensorMap& wa, const CUten
   return cuda_status(cudaGetLastError());
 }
 
-PaletteTables palette_tables(const uint8_t* pal, const uint8_t* code_len, bool* mixed) {
-  PaletteTables t;
-  uint32_t w[4] = {0, 0, 0, 0}, b7[4] = {0, 0, 0, 0};
-  int seen0 = 0, seen1 = 0;
-  for (int i = 0; i < 16; ++i) {
-    w[i / 4] |= static_cast<uint32_t>(pal[i] | 0x80u) << (8 * (i % 4));
-    b7[i / 4] |= static_cast<uint32_t>(0xBFu | ((pal[i] >> 7) << 6)) << (8 * (i % 4));
-    if (!code_len || code_len[i]) {
-      if (pal[i] & 0x80) seen1 = 1;
-      else seen0 = 1;
-    }
-  }
-  t.lo0 = w[0];
-  t.lo1 = w[1];
-  t.hi0 = w[2];
-  t.hi1 = w[3];
-  t.b7lo0 = b7[0];
-  t.b7lo1 = b7[1];
-  t.b7hi0 = b7[2];
-  t.b7hi1 = b7[3];
-  *mixed = seen0 && seen1;
-  t.keep = seen1 ? 0xFFFFFFFFu : 0x7F7F7F7Fu;
-  return t;
-}
 
 }  // namespace
 

@@ -71,6 +71,9 @@ uw_status check_matrix(const uw_matrix* m);
 
 // Kernel launchers (asynchronous).
 uw_status launch_decode(const uw_matrix* m, int mode, void* out, uint32_t* status, cudaStream_t s);
+// Full decode of rows[0..n_rows) (device int32) into out [n_rows, cols] BF16.
+uw_status launch_decode_rows(const uw_matrix* m, const int32_t* rows, int64_t n_rows, void* out, uint32_t* status,
+                             cudaStream_t s);
 enum Loader { kLoaderBF16 = 0, kLoaderEXP8 = 1, kLoaderIDX4 = 2, kLoaderPACK = 3 };
 struct GemmArgs {
   int loader = kLoaderIDX4;

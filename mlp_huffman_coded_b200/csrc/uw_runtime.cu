@@ -215,4 +215,10 @@ extern "C" uw_status uw_transcode_palette(const uw_matrix* m, uint8_t* out, void
   return decode_entry(m, 2, out, ws, ws_bytes, stream);
 }
 
+extern "C" uw_status uw_decode_rows(const uw_matrix* m, const int32_t* rows, int32_t n_rows, uint16_t* out,
+                                    void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < kWsHeader || !aligned16(ws)) return ws ? UW_ERR_WORKSPACE_TOO_SMALL : UW_ERR_INVALID_ARG;
+  return launch_decode_rows(m, rows, n_rows, out, static_cast<uint32_t*>(ws), static_cast<cudaStream_t>(stream));
+}
+
 extern "C" uint64_t uw_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -72,6 +72,7 @@ _SIGS = {
     "uw_decode_full": (C.c_int, [C.POINTER(Matrix), _P, _P, C.c_size_t, _P]),
     "uw_decode_exponent_only": (C.c_int, [C.POINTER(Matrix), _P, _P, C.c_size_t, _P]),
     "uw_transcode_palette": (C.c_int, [C.POINTER(Matrix), _P, _P, C.c_size_t, _P]),
+    "uw_decode_rows": (C.c_int, [C.POINTER(Matrix), _P, C.c_int32, _P, _P, C.c_size_t, _P]),
     "uw_gemm_direct_palette": (C.c_int, [C.POINTER(Matrix), _P, C.c_int32, _P, _P, C.c_size_t, _P]),
     "uw_gemm_direct_palette_general_lookup": (C.c_int, [C.POINTER(Matrix), _P, C.c_int32, _P, _P,
                                                         C.c_size_t, _P]),
@@ -325,6 +326,12 @@ def decode_full(dm: DeviceMatrix, out, ws: Workspace, stream=None):
 def decode_exponent_only(dm: DeviceMatrix, out, ws: Workspace, stream=None):
     _check(lib().uw_decode_exponent_only(C.byref(dm.mat), _ptr(out), ws.ptr, ws.nbytes, _stream(stream)),
            "uw_decode_exponent_only")
+
+
+def decode_rows(dm: DeviceMatrix, rows, out, ws: Workspace, stream=None):
+    """out[i] = row rows[i] of W (rows: device int32 tensor)."""
+    _check(lib().uw_decode_rows(C.byref(dm.mat), _ptr(rows), rows.numel(), _ptr(out), ws.ptr, ws.nbytes,
+                                _stream(stream)), "uw_decode_rows")
 
 
 def transcode_palette(dm: DeviceMatrix, out, ws: Workspace, stream=None):

@@ -166,3 +166,49 @@ def test_prefixes_pointing_outside_the_store_are_reported_not_faulted():
     uw.gemm(dm, uw.PIPE_TRANSCODE, x, y, wsg)
     assert wsg.status() == uw.UW_ERR_CORRUPT
     assert wsg.status() == uw.UW_OK
+
+
+def _gather(dm, rows):
+    import torch
+    ws = uw.Workspace(256)
+    out = empty_bf16(len(rows), dm.cols)
+    uw.decode_rows(dm, torch.tensor(rows, dtype=torch.int32, device="cuda"), out, ws)
+    return ws, to_host_u16(out).reshape(len(rows), dm.cols)
+
+
+@pytest.mark.parametrize("rows,cols,chunk_groups,rate", [
+    (300, 640, 3, 2e-2),    # 10 groups per row: chunks straddle rows
+    (257, 4096, 4, 1e-3),   # chunks aligned with rows, ragged last row tile
+    (64, 1024, 16, 0.0),    # one chunk per row
+])
+def test_decode_rows_is_the_rows_of_w(rows, cols, chunk_groups, rate):
+    """Embedding lookup: every requested row (repeats, first, last, in any
+    order) comes back bit for bit, verbatim groups included."""
+    w = synth.weight_matrix(rows, cols, 0.02, rate, 300.0, 101)
+    dm = device_matrix(w, chunk_groups=chunk_groups, direct=False)
+    ids = [rows - 1, 0, 5, 5, rows // 2, 1, rows - 1] + list(np.random.default_rng(102).integers(0, rows, 40))
+    ws, got = _gather(dm, ids)
+    ws.check("decode rows")
+    assert np.array_equal(got, w[ids])
+
+
+def test_decode_rows_embedding_table():
+    """A vocabulary-sized table (32000 x 4096, the shape of a 32K-token
+    embedding): 512 random token ids."""
+    w = synth.weight_matrix(32000, 4096, 0.02, 1e-4, 100.0, 103)
+    dm = device_matrix(w, direct=False)
+    ids = list(np.random.default_rng(104).integers(0, 32000, 512))
+    ws, got = _gather(dm, ids)
+    ws.check("decode rows")
+    assert np.array_equal(got, w[ids])
+
+
+def test_decode_rows_outside_the_matrix_are_reported():
+    w = synth.weight_matrix(100, 512, 0.02, 1e-3, 100.0, 105)
+    dm = device_matrix(w, direct=False)
+    ws, got = _gather(dm, [3, 100, -1, 99])
+    with pytest.raises(uw.UwError) as e:
+        ws.check("decode rows")
+    assert e.value.status == uw.UW_ERR_INVALID_ARG
+    assert np.array_equal(got[0], w[3]) and np.array_equal(got[3], w[99])
+    assert not got[1].any() and not got[2].any()
