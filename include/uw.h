@@ -279,6 +279,42 @@ UW_API uw_status uw_selftest_bounded_wait(void* workspace, size_t workspace_byte
                                           void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Load-time compression on the GPU (section "Four ways to use compressed
+ * weights": the direct palette is prepared when the model is loaded; section
+ * "How to compress model weights effectively": the format)
+ * ------------------------------------------------------------------------- */
+
+/* Device workspace bytes of the two calls below for a [rows, cols] matrix
+ * (0 for an unsupported shape): about 13 bytes per 64-element group. */
+UW_API size_t uw_encode_gpu_workspace_bytes(int64_t rows, int64_t cols);
+
+/* uw_build_palette_codebook for a device-resident W (device BF16 [rows,
+ * cols], 16-byte aligned): the exponent histogram and the per-index counts
+ * over non-verbatim groups are computed on the GPU; the palette and the
+ * Huffman code are chosen on the host from those counts by the same
+ * routines as the host call, so *out is identical to it.  Synchronizes
+ * `stream` (twice).  Errors as uw_build_palette_codebook, plus
+ * UW_ERR_WORKSPACE_TOO_SMALL, UW_ERR_NO_DEVICE, UW_ERR_CUDA. */
+UW_API uw_status uw_build_palette_codebook_gpu(const uint16_t* w, int64_t rows, int64_t cols,
+                                               uw_codebook* out, void* workspace,
+                                               size_t workspace_bytes, void* stream);
+
+/* uw_encode for a device-resident W: the same *L and the same sm, stream,
+ * chunk_bit_off, vflags, vprefix and verbatim bytes as the host call, written
+ * to device buffers (16-byte aligned, sized from *L as for uw_encode).  With
+ * every output NULL only *L is filled.  Each call runs the group pass and
+ * synchronizes `stream` to read the totals; the writing call synchronizes
+ * again at its end.  Errors as uw_encode (UW_ERR_CORRUPT for a codebook that
+ * leaves a used palette index without a code, UW_ERR_UNSUPPORTED_SHAPE for
+ * 2^32 or more stream bits), plus UW_ERR_WORKSPACE_TOO_SMALL,
+ * UW_ERR_NO_DEVICE, UW_ERR_CUDA. */
+UW_API uw_status uw_encode_gpu(const uint16_t* w, int64_t rows, int64_t cols, const uw_codebook* cb,
+                               int32_t chunk_groups, uw_layout* L, uint8_t* sm, uint32_t* stream,
+                               uint32_t* chunk_bit_off, uint32_t* vflags, uint32_t* vprefix,
+                               uint16_t* verbatim, void* workspace, size_t workspace_bytes,
+                               void* cuda_stream);
+
+/* ---------------------------------------------------------------------------
  * Preprocessing kernels (section "Four ways to use compressed weights")
  * ------------------------------------------------------------------------- */
 

@@ -24,8 +24,8 @@ LIB = os.path.join(PKG, "libuw.so")
 BUILD_DIR = os.path.join(PKG, "_build")
 
 SOURCES = ["uw_host.cpp", "uw_runtime.cu", "uw_decode.cu", "uw_pack.cu", "uw_gemm.cu", "uw_autotune.cu",
-           "uw_noalloc.cu", "uw_selftest.cu"]
-HEADERS = ["uw_device.cuh", "uw_internal.h"]
+           "uw_noalloc.cu", "uw_selftest.cu", "uw_encode_gpu.cu"]
+HEADERS = ["uw_device.cuh", "uw_internal.h", "uw_codebook.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden",

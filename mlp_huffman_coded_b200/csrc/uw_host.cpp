@@ -17,6 +17,7 @@
 #include <vector>
 
 #include "uw.h"
+#include "uw_codebook.h"
 
 namespace {
 
@@ -126,6 +127,34 @@ void canonical(const uint8_t* len, uint16_t* code) {
 
 }  // namespace
 
+namespace uw {
+
+void choose_palette(const uint64_t* hist, uint8_t* palette) {
+  std::array<int, 256> order;
+  for (int e = 0; e < 256; ++e) order[e] = e;
+  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
+    if (hist[a] != hist[b]) return hist[a] > hist[b];
+    return a < b;
+  });
+  for (int i = 0; i < kPal; ++i) palette[i] = static_cast<uint8_t>(order[i]);
+}
+
+void finish_codebook(uw_codebook* cb) {
+  huffman_lengths(cb->freq, cb->code_len);
+  canonical(cb->code_len, cb->code);
+  int ns = 0, ml = 0;
+  for (int i = 0; i < kPal; ++i) {
+    ns += cb->code_len[i] > 0;
+    ml = std::max<int>(ml, cb->code_len[i]);
+  }
+  cb->n_symbols = static_cast<uint8_t>(ns);
+  cb->max_len = static_cast<uint8_t>(ml);
+}
+
+bool encode_shape_ok(int64_t rows, int64_t cols) { return shape_ok(rows, cols); }
+
+}  // namespace uw
+
 extern "C" uw_status uw_build_palette_codebook(const uint16_t* w, int64_t rows, int64_t cols,
                                                 uw_codebook* out) {
   if (!w || !out) return UW_ERR_INVALID_ARG;
@@ -142,15 +171,9 @@ extern "C" uw_status uw_build_palette_codebook(const uint16_t* w, int64_t rows, 
   std::array<uint64_t, 256> hist{};
   for (int t = 0; t < nt; ++t)
     for (int e = 0; e < 256; ++e) hist[e] += part_hist[t][e];
-  std::array<int, 256> order;
-  for (int e = 0; e < 256; ++e) order[e] = e;
-  std::stable_sort(order.begin(), order.end(), [&](int a, int b) {
-    if (hist[a] != hist[b]) return hist[a] > hist[b];
-    return a < b;
-  });
   uw_codebook cb;
   std::memset(&cb, 0, sizeof(cb));
-  for (int i = 0; i < kPal; ++i) cb.palette[i] = static_cast<uint8_t>(order[i]);
+  uw::choose_palette(hist.data(), cb.palette);
   auto pm = palette_map(cb.palette);
   // frequencies over non-verbatim groups only
   std::vector<std::array<uint64_t, kPal>> part_freq(nt);
@@ -167,15 +190,7 @@ extern "C" uw_status uw_build_palette_codebook(const uint16_t* w, int64_t rows, 
   });
   for (int t = 0; t < nt; ++t)
     for (int i = 0; i < kPal; ++i) cb.freq[i] += part_freq[t][i];
-  huffman_lengths(cb.freq, cb.code_len);
-  canonical(cb.code_len, cb.code);
-  int ns = 0, ml = 0;
-  for (int i = 0; i < kPal; ++i) {
-    ns += cb.code_len[i] > 0;
-    ml = std::max<int>(ml, cb.code_len[i]);
-  }
-  cb.n_symbols = static_cast<uint8_t>(ns);
-  cb.max_len = static_cast<uint8_t>(ml);
+  uw::finish_codebook(&cb);
   *out = cb;
   return UW_OK;
 }

@@ -63,6 +63,10 @@ _SIGS = {
     "uw_encode": (C.c_int, [_P, C.c_int64, C.c_int64, C.POINTER(Codebook), C.c_int32, C.POINTER(Layout),
                             _P, _P, _P, _P, _P, _P]),
     "uw_validate": (C.c_int, [C.POINTER(Matrix)]),
+    "uw_encode_gpu_workspace_bytes": (C.c_size_t, [C.c_int64, C.c_int64]),
+    "uw_build_palette_codebook_gpu": (C.c_int, [_P, C.c_int64, C.c_int64, C.POINTER(Codebook), _P, C.c_size_t, _P]),
+    "uw_encode_gpu": (C.c_int, [_P, C.c_int64, C.c_int64, C.POINTER(Codebook), C.c_int32, C.POINTER(Layout),
+                                _P, _P, _P, _P, _P, _P, _P, C.c_size_t, _P]),
     "uw_direct_pack_offsets": (C.c_int, [C.POINTER(Layout), _P, _P, C.POINTER(C.c_uint64)]),
     "uw_selftest_bounded_wait": (C.c_int, [_P, C.c_size_t, C.c_uint32, _P]),
     "uw_pack_direct_palette": (C.c_int, [C.POINTER(Matrix), _P, _P, _P]),
@@ -173,13 +177,9 @@ class HostEncoded:
         return m
 
     def pack_offsets(self):
-        """Direct-palette record offsets (16-byte units) and total bytes."""
-        n_tiles = -(-self.rows // 128) * (self.cols // 64)
-        off = np.empty(n_tiles + 1, np.uint32)
-        total = C.c_uint64()
-        _check(lib().uw_direct_pack_offsets(C.byref(self.layout), _ptr(self.vflags), _ptr(off), C.byref(total)),
-               "uw_direct_pack_offsets")
-        return off, int(total.value)
+        """Direct-palette pack offsets (verbatim rows before each tile) and
+        total pack bytes."""
+        return _pack_offsets(self.layout, self.vflags)
 
     def compressed_bytes(self, form: str = "huffman") -> int:
         meta = self.vflags.nbytes + self.vprefix.nbytes + self.verbatim.nbytes
@@ -188,6 +188,16 @@ class HostEncoded:
         if form == "palette":
             return self.sm.nbytes + self.rows * self.cols // 2 + meta
         raise ValueError(form)
+
+
+def _pack_offsets(layout: Layout, vflags: np.ndarray):
+    n_tiles = -(-int(layout.rows) // 128) * (int(layout.cols) // 64)
+    off = np.empty(n_tiles + 1, np.uint32)
+    total = C.c_uint64()
+    vflags = np.ascontiguousarray(vflags, dtype=np.uint32)
+    _check(lib().uw_direct_pack_offsets(C.byref(layout), _ptr(vflags), _ptr(off), C.byref(total)),
+           "uw_direct_pack_offsets")
+    return off, int(total.value)
 
 
 def build_codebook(w: np.ndarray) -> Codebook:
@@ -288,6 +298,56 @@ class DeviceMatrix:
     def cols(self):
         return int(self.mat.L.cols)
 
+    @classmethod
+    def encode_on_device(cls, w, chunk_groups: int = 4, cb: Codebook | None = None, stream=None):
+        """Compress a device-resident BF16 matrix on the GPU (torch int16 /
+        bfloat16 tensor [rows, cols]): uw_build_palette_codebook_gpu and
+        uw_encode_gpu, whose outputs equal the host encoder's byte for
+        byte.  No host copy of W is made."""
+        import torch
+        w = w.contiguous()
+        rows, cols = w.shape
+        dev = w.device
+        wsn = int(lib().uw_encode_gpu_workspace_bytes(rows, cols))
+        if wsn == 0:
+            raise UwError(UW_ERR_UNSUPPORTED_SHAPE, "uw_encode_gpu_workspace_bytes")
+        ws = torch.empty(wsn, dtype=torch.uint8, device=dev)
+        st = _stream(stream)
+        if cb is None:
+            cb = Codebook()
+            _check(lib().uw_build_palette_codebook_gpu(w.data_ptr(), rows, cols, C.byref(cb), ws.data_ptr(), wsn, st),
+                   "uw_build_palette_codebook_gpu")
+        L = Layout()
+        f = lib().uw_encode_gpu
+        _check(f(w.data_ptr(), rows, cols, C.byref(cb), chunk_groups, C.byref(L), None, None, None, None, None, None,
+                 ws.data_ptr(), wsn, st), "uw_encode_gpu (sizes)")
+        self = cls.__new__(cls)
+        self.enc = None
+        self.device = dev
+        self.sm = torch.empty(rows * cols, dtype=torch.uint8, device=dev)
+        self.stream = torch.empty(int(L.stream_words), dtype=torch.int32, device=dev)
+        self.chunk_bit_off = torch.empty(int(L.n_chunks) + 1, dtype=torch.int32, device=dev)
+        self.vflags = torch.empty(rows * int(L.words_per_row), dtype=torch.int32, device=dev)
+        self.vprefix = torch.empty(rows * int(L.words_per_row) + 1, dtype=torch.int32, device=dev)
+        self.verbatim = torch.empty(int(L.n_verbatim) * 64, dtype=torch.int16, device=dev) if L.n_verbatim else None
+        _check(f(w.data_ptr(), rows, cols, C.byref(cb), chunk_groups, C.byref(L), self.sm.data_ptr(),
+                 self.stream.data_ptr(), self.chunk_bit_off.data_ptr(), self.vflags.data_ptr(),
+                 self.vprefix.data_ptr(), _ptr(self.verbatim), ws.data_ptr(), wsn, st), "uw_encode_gpu")
+        self.idx4 = None
+        self.mat = Matrix()
+        self.mat.L = L
+        self.mat.cb = cb
+        self.mat.sm, self.mat.stream = self.sm.data_ptr(), self.stream.data_ptr()
+        self.mat.chunk_bit_off = self.chunk_bit_off.data_ptr()
+        self.mat.vflags, self.mat.vprefix = self.vflags.data_ptr(), self.vprefix.data_ptr()
+        self.mat.verbatim = self.verbatim.data_ptr() if self.verbatim is not None else None
+        self.mat.idx4 = None
+        self.mat.pack = None
+        self.mat.pack_off = None
+        self.pack = None
+        self.pack_off = None
+        return self
+
     def prepare_direct_palette(self, ws: Workspace, stream=None, keep_idx4: bool = True):
         """Load-time preparation of the direct-palette form: transcode to 4-bit
         palette indices, then gather sm + indices + verbatim rows into one
@@ -296,7 +356,10 @@ class DeviceMatrix:
         self.idx4 = torch.empty(self.rows * self.cols // 2, dtype=torch.uint8, device=self.device)
         transcode_palette(self, self.idx4, ws, stream)
         self.mat.idx4 = self.idx4.data_ptr()
-        off, nbytes = self.enc.pack_offsets()
+        if self.enc is not None:
+            off, nbytes = self.enc.pack_offsets()
+        else:
+            off, nbytes = _pack_offsets(self.mat.L, self.vflags.cpu().numpy().view(np.uint32))
         self.pack_off = torch.from_numpy(off.view(np.int32)).to(self.device)
         self.pack = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         _check(lib().uw_pack_direct_palette(C.byref(self.mat), self.pack_off.data_ptr(), self.pack.data_ptr(),
