@@ -637,7 +637,7 @@ def run_stack_time_case(args, local):
     matrices, per-layer sigma uniform in [0.01, 0.05], 1e-3 outliers x100) at
     batch 1 and 64, measured end to end: every layer's weights are drawn on
     the GPU (synth.stack_layer_device: the stack recipe with torch's
-    generator), host-encoded and packed on the GPU, each matrix's pipeline is
+    generator), compressed and packed on the GPU, each matrix's pipeline is
     picked by uw_autotune, and one timed step is one uw_mlp_stack call (all
     GEMMs of all layers, back to back on one stream).  L2 is flushed before
     each step (the packed stack is ~9 GB anyway).  Beside it: the same
@@ -660,8 +660,7 @@ def run_stack_time_case(args, local):
         ws_bf16 = synth.stack_layer_device(layer, dev)
         triple, ch = [], []
         for w in ws_bf16:
-            enc = uw.encode(w.cpu().numpy().view(np.uint16))
-            dm = uw.DeviceMatrix(enc, device=dev).prepare_direct_palette(ws0, keep_idx4=False)
+            dm = uw.DeviceMatrix.encode_on_device(w).prepare_direct_palette(ws0, keep_idx4=False)
             ws0.check("prepare")
             rows, cols = int(dm.mat.L.rows), int(dm.mat.L.cols)
             if xa is None or xa.shape[1] < cols or ya.shape[1] < rows:
@@ -671,7 +670,6 @@ def run_stack_time_case(args, local):
             c, _ = uw.autotune(dm, batches, 3, xa[:, :cols].contiguous(), ya, wsa, flush=flush)
             wsa.check("autotune")
             del wsa
-            dm.enc = None  # host copy no longer needed
             pack_bytes += dm.direct_palette_bytes()
             triple.append(dm)
             ch.append([int(v) for v in c])
@@ -709,6 +707,57 @@ def run_stack_time_case(args, local):
     return 0
 
 
+def run_shapes_case(args, local):
+    """The scheme on the non-MLP matrices of a Llama-3.1-8B-shaped model
+    (weights drawn on the GPU with the MLP recipe: N(0, 0.02), 1e-4
+    outliers x100; compressed on the GPU): direct-palette GEMM vs
+    torch.matmul BF16 for q/o (4096 x 4096), k/v (1024 x 4096) and the
+    output projection (128256 x 4096) at batch 1, 8, 64, L2 flushed before
+    each call; and the embedding lookup of 64 tokens from a compressed
+    128256 x 4096 table (uw_decode_rows) vs torch.index_select on BF16."""
+    import torch
+    from mlp_huffman_coded_b200 import synth, uw
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    flush = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+    ws0 = uw.Workspace(256, device=dev)
+    peaks, src = measured_peaks()
+    hbm = peaks.get("hbm_gbs", HBM_FALLBACK_GBS)
+    shapes = [("q_proj/o_proj", 4096, 4096, 130), ("k_proj/v_proj", 1024, 4096, 131),
+              ("lm_head", 128256, 4096, 132)]
+    for name, rows, cols, seed in shapes:
+        w = synth.weight_matrix_device(rows, cols, SIGMA, OUTLIER_RATE, OUTLIER_SCALE, seed, dev)
+        dm = uw.DeviceMatrix.encode_on_device(w).prepare_direct_palette(ws0, keep_idx4=False)
+        ws0.check("prepare")
+        wb = w.view(torch.bfloat16)
+        for B in (1, 8, 64):
+            x = torch.from_numpy(synth.activations(B, cols, 3).view(np.int16)).to(dev)
+            y = torch.empty(B, rows, dtype=torch.int16, device=dev)
+            ws = uw.Workspace(uw.workspace_bytes(dm, uw.PIPE_DIRECT, B), device=dev)
+            med, _ = _timed(lambda: uw.gemm_direct_palette(dm, x, y, ws), flush, args.steps, args.warmup, dev)
+            ws.check("gemm")
+            xb = x.view(torch.bfloat16)
+            tmed, _ = _timed(lambda: xb @ wb.T, flush, args.steps, args.warmup, dev)
+            nbytes = dm.direct_palette_bytes()
+            print(json.dumps({"case": "shapes", "matrix": f"{name} {rows}x{cols}", "batch": B,
+                              "direct_palette_us": med, "torch_bf16_us": tmed, "speedup_vs_bf16": tmed / med,
+                              "packed_bytes": nbytes, "bf16_bytes": rows * cols * 2,
+                              "packed_gbs": nbytes / med / 1e3, "hbm_frac": nbytes / med / 1e3 / hbm,
+                              "hbm_peak_gbs": hbm, "peak_source": src}), flush=True)
+            del ws
+        if name == "lm_head":
+            ids = torch.from_numpy(np.random.default_rng(5).integers(0, rows, 64).astype(np.int32)).to(dev)
+            out = torch.empty(64, cols, dtype=torch.int16, device=dev)
+            med, _ = _timed(lambda: uw.decode_rows(dm, ids, out, ws0), flush, args.steps, args.warmup, dev)
+            ws0.check("decode rows")
+            tmed, _ = _timed(lambda: torch.index_select(wb, 0, ids), flush, args.steps, args.warmup, dev)
+            print(json.dumps({"case": "shapes", "matrix": f"embedding {rows}x{cols}", "tokens": 64,
+                              "decode_rows_us": med, "torch_index_select_us": tmed}), flush=True)
+        del dm, w, wb
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -720,19 +769,22 @@ def main(argv=None):
     ap.add_argument("--ref-fraction", type=float, default=1 / 16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--layers", type=int, default=32, help="stack / stack-time cases: layers to use")
-    ap.add_argument("--case", default="block", choices=["block", "gemm", "decode", "sweep", "stack", "stack-time"],
+    ap.add_argument("--case", default="block",
+                    choices=["block", "gemm", "decode", "sweep", "stack", "stack-time", "shapes"],
                     help="gemm: one 14336x4096 matrix through --pipeline (profiling unit); decode: the three "
                          "decoders on it; sweep: pipelines x batch 1..512 x block matrices + autotune; "
                          "stack: compressed size of the 32-layer stack (host only); stack-time: decode-step "
-                         "MLP time of the --layers-layer stack (one uw_mlp_stack call) at batch 1 and 64")
+                         "MLP time of the --layers-layer stack (one uw_mlp_stack call) at batch 1 and 64; shapes: "
+                         "attention / output-projection GEMMs and the embedding lookup")
     ap.add_argument("--pipeline", default="direct", choices=["full", "exponent", "transcode", "direct", "bf16"])
     ap.add_argument("--no-flush", action="store_true", help="gemm case: leave L2 warm between calls")
     args = ap.parse_args(argv)
     if args.steps is None:
         args.steps = 20 if args.impl == "reference" else {"gemm": 100, "decode": 20, "sweep": 10,
-                                                         "stack-time": 20}.get(args.case, 3000)
+                                                         "stack-time": 20, "shapes": 20}.get(args.case, 3000)
     if args.warmup is None:
-        args.warmup = 3 if args.impl == "reference" or args.case in ("sweep", "decode", "stack-time") else 20
+        args.warmup = 3 if args.impl == "reference" or args.case in ("sweep", "decode", "stack-time",
+                                                                       "shapes") else 20
     if args.case == "stack":
         return run_stack_case(args)
     world, rank, local = dist_init()
@@ -747,6 +799,8 @@ def main(argv=None):
             return run_sweep_case(args, local)
         if args.case == "stack-time":
             return run_stack_time_case(args, local)
+        if args.case == "shapes":
+            return run_shapes_case(args, local)
         return run_gpu(args, world, rank, local)
     finally:
         if world > 1:

@@ -30,6 +30,9 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "uw_device.cuh"
 #include "uw_internal.h"
@@ -41,6 +44,10 @@ namespace {
 constexpr int kLutBits = 11;
 constexpr int kLutSize = 1 << kLutBits;
 constexpr int kStageBudget = 48 * 1024;  // per block: index stage + group info
+// Row gather: each warp first copies the stream words of its chunks into
+// shared memory with coalesced loads (a few warps decode a few rows, so the
+// lanes' dependent refills would otherwise each wait for HBM).
+constexpr int kRowStreamWords = 2048;
 
 enum DecodeMode { kFull = 0, kExp8 = 1, kIdx4 = 2 };
 
@@ -85,21 +92,33 @@ struct DecodeTables {
 // lut: kLutSize words of scratch (the first code of each prefix, sym |
 // len << 4, len 0 = longer than the table), needed only while building.
 __device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables& t, uint16_t* lut) {
-  if (threadIdx.x == 0) {
-    for (int l = 0; l <= 16; ++l) t.count[l] = 0;
-    for (int i = 0; i < 16; ++i)
-      if (p.code_len[i]) ++t.count[p.code_len[i]];
-    uint32_t code = 0, pos = 0;
-    for (int l = 1; l <= 16; ++l) {
-      t.first[l] = code;
-      t.offset[l] = pos;
-      code = (code + t.count[l]) << 1;
-      pos += t.count[l];
+  // warp 0: code counts per length, the canonical first codes, and the
+  // symbols in (length, index) order (each symbol placed at its rank in
+  // that order)
+  if (threadIdx.x < 32) {
+    const int i = threadIdx.x;
+    const int li = i < 16 ? p.code_len[i] : 0;
+    if (i <= 16) t.count[i] = 0;
+    __syncwarp();
+    if (i < 16 && li > 0) {
+      int rank = 0;
+      for (int j = 0; j < 16; ++j) {
+        const int lj = p.code_len[j];
+        rank += (lj > 0 && (lj < li || (lj == li && j < i))) ? 1 : 0;
+      }
+      t.sorted[rank] = static_cast<uint8_t>(i);
+      atomicAdd(&t.count[li], 1u);
     }
-    int k = 0;
-    for (int l = 1; l <= 15; ++l)
-      for (int i = 0; i < 16; ++i)
-        if (p.code_len[i] == l) t.sorted[k++] = static_cast<uint8_t>(i);
+    __syncwarp();
+    if (i == 0) {
+      uint32_t code = 0, pos = 0;
+      for (int l = 1; l <= 16; ++l) {
+        t.first[l] = code;
+        t.offset[l] = pos;
+        code = (code + t.count[l]) << 1;
+        pos += t.count[l];
+      }
+    }
   }
   __syncthreads();
   const int lim = p.max_len < kLutBits ? p.max_len : kLutBits;
@@ -160,8 +179,10 @@ __device__ __forceinline__ uint32_t stage_word(int lane, int w, int cg, int umas
 // their slots, 8 words each) and records every group's source in info[]:
 // -1 coded, >= 0 verbatim slot, -2 unreadable verbatim slot (written as
 // zeros), -3 past the matrix.
+// sbuf (may be NULL): stream words [sbase, sbase + sn) in shared memory.
 __device__ __forceinline__ void decode_chunk(const DecodeParams& p, const DecodeTables& t, int64_t c, int lane,
-                                             uint32_t* stage, int32_t* info, int umask) {
+                                             uint32_t* stage, int32_t* info, int umask, const uint32_t* sbuf,
+                                             int64_t sbase, int64_t sn) {
   const int cg = p.chunk_groups;
   const int64_t g0 = c * cg;
   const int64_t g1 = min(g0 + cg, p.n_groups);
@@ -195,10 +216,14 @@ __device__ __forceinline__ void decode_chunk(const DecodeParams& p, const Decode
   }
   const uint32_t b0 = __ldg(p.off + c), b1 = __ldg(p.off + c + 1);
   const int64_t last_word = p.stream_words - 1;
+  auto fetch = [&](int64_t i) -> uint32_t {
+    const int64_t k = i - sbase;
+    return (sbuf && k >= 0 && k < sn) ? sbuf[k] : __ldg(p.stream + min(i, last_word));
+  };
   int64_t wi = b0 >> 5;
-  uint32_t w0 = __ldg(p.stream + min(wi, last_word));
-  uint32_t w1 = __ldg(p.stream + min(wi + 1, last_word));
-  uint32_t w2 = __ldg(p.stream + min(wi + 2, last_word));
+  uint32_t w0 = fetch(wi);
+  uint32_t w1 = fetch(wi + 1);
+  uint32_t w2 = fetch(wi + 2);
   wi += 3;
   int bp = static_cast<int>(b0 & 31);
   uint32_t consumed = 0;
@@ -231,7 +256,7 @@ __device__ __forceinline__ void decode_chunk(const DecodeParams& p, const Decode
     consumed += static_cast<uint32_t>(len);
     const bool cross = bp >= 32;
     uint32_t nw = 0;
-    if (cross) nw = __ldg(p.stream + min(wi, last_word));
+    if (cross) nw = fetch(wi);
     bp -= cross ? 32 : 0;
     w0 = cross ? w1 : w0;
     w1 = cross ? w2 : w1;
@@ -354,6 +379,7 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
   const int cg = p.chunk_groups;
   uint32_t* stage = dsm + warp * (256 * cg);
   int32_t* info = reinterpret_cast<int32_t*>(dsm + W * 256 * cg) + warp * 32 * cg;
+  uint32_t* sbuf = ROWS ? dsm + W * 288 * cg + warp * kRowStreamWords : nullptr;
   const int units = 2 * cg;
   const int umask = min(units & -units, 8) - 1;
   for (int64_t it = static_cast<int64_t>(blockIdx.x) * W + warp; it < p.n_items;
@@ -385,8 +411,18 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
       g_hi = min(c_end * cg, rg1);
       og0 = i * p.gpr + (g_lo - rg0);
     }
+    int64_t sbase = 0, sn = 0;
+    if (ROWS && !zero) {
+      // the stream words of chunks [c_first, c_end), plus the three-word
+      // window's overrun, into the warp's buffer
+      sbase = __ldg(p.off + c_first) >> 5;
+      sn = min(static_cast<int64_t>((__ldg(p.off + c_end) >> 5) + 3 - sbase), static_cast<int64_t>(kRowStreamWords));
+      const int64_t last_word = p.stream_words - 1;
+      for (int64_t k = lane; k < sn; k += 32) sbuf[k] = __ldg(p.stream + min(sbase + k, last_word));
+      __syncwarp();
+    }
     const int64_t c = c_first + lane;
-    if (c < c_end && !zero) decode_chunk(p, t, c, lane, stage, info, umask);
+    if (c < c_end && !zero) decode_chunk(p, t, c, lane, stage, info, umask, sbuf, sbase, sn);
     __syncwarp();
     emit_groups<MODE>(p, stage, info, umask, c_first * cg, static_cast<int>(g_lo - c_first * cg),
                       static_cast<int>(g_hi - c_first * cg), og0, zero);
@@ -429,19 +465,46 @@ uw_status fill_params(const uw_matrix* m, void* out, uint32_t* status, DecodePar
 // most 8.
 int warps_per_block(int cg) { return std::max(1, std::min(8, kStageBudget / (cg * 1152))); }
 
+// Per device: the kernel's shared-memory opt-in (set once: the call is not
+// free and may wait for the device) and its resident blocks per SM for each
+// dynamic shared-memory size (looked up once).
+template <int MODE, bool ROWS>
+uw_status resident_blocks(int dev, size_t smem, int threads, int* per_sm) {
+  static std::mutex mu;
+  static std::map<std::pair<int, size_t>, int> cache;
+  static bool attr_set[64] = {};
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find({dev, smem});
+  if (it != cache.end()) {
+    *per_sm = it->second;
+    return UW_OK;
+  }
+  if (!attr_set[dev & 63]) {
+    if (cudaFuncSetAttribute(decode_kernel<MODE, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kStageBudget + 8 * kRowStreamWords * 4) != cudaSuccess)
+      return UW_ERR_CUDA;
+    attr_set[dev & 63] = true;
+  }
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_kernel<MODE, ROWS>, threads, smem) != cudaSuccess)
+    return UW_ERR_CUDA;
+  cache[{dev, smem}] = n;
+  *per_sm = n;
+  return UW_OK;
+}
+
 template <int MODE, bool ROWS>
 uw_status launch(const DecodeParams& p, const DeviceInfo& dev, cudaStream_t s) {
   if (p.n_items <= 0) return UW_OK;
   const int W = warps_per_block(p.chunk_groups);
   // (also the table build's kLutSize-word scratch)
-  const size_t smem = std::max<size_t>(static_cast<size_t>(W) * p.chunk_groups * 1152, kLutSize * 2);
-  if (cudaFuncSetAttribute(decode_kernel<MODE, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStageBudget) !=
-      cudaSuccess)
-    return UW_ERR_CUDA;
+  const size_t smem = std::max<size_t>(static_cast<size_t>(W) * p.chunk_groups * 1152, kLutSize * 2) +
+                      (ROWS ? static_cast<size_t>(W) * kRowStreamWords * 4 : 0);
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return UW_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_kernel<MODE, ROWS>, 32 * W, smem) !=
-      cudaSuccess)
-    return UW_ERR_CUDA;
+  const uw_status st = resident_blocks<MODE, ROWS>(device, smem, 32 * W, &per_sm);
+  if (st != UW_OK) return st;
   const int64_t blocks_needed = (p.n_items + W - 1) / W;
   const int64_t resident = static_cast<int64_t>(dev.sm_count) * std::max(1, per_sm);
   const int grid = static_cast<int>(std::min(blocks_needed, resident));

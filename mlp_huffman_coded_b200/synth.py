@@ -24,6 +24,7 @@ __all__ = [
     "stack_sigmas",
     "stack_layer",
     "stack_layer_device",
+    "weight_matrix_device",
 ]
 
 
@@ -121,27 +122,33 @@ def stack_layer(layer: int, n_layers: int = 32, d_model: int = 4096, ffn: int = 
             weight_matrix(d_model, ffn, sigma, outlier_rate, outlier_scale, seed + 2))
 
 
+def weight_matrix_device(rows: int, cols: int, sigma: float, outlier_rate: float, outlier_scale: float,
+                         seed: int, device):
+    """`weight_matrix`'s recipe drawn on a torch device with torch's
+    generator seeded `seed` (so the values differ from `weight_matrix`'s):
+    N(0, sigma), entries below `outlier_rate` in a uniform draw scaled by
+    `outlier_scale`, RNE to BF16.  Returns an int16 tensor of the BF16
+    patterns.  For the timed cases that need many or large matrices
+    quickly; every parity case uses `weight_matrix`."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    w = torch.randn(rows, cols, generator=g, device=device, dtype=torch.float32) * sigma
+    if outlier_rate > 0:
+        mask = torch.rand(rows, cols, generator=g, device=device) < outlier_rate
+        w = torch.where(mask, w * outlier_scale, w)
+    return w.to(torch.bfloat16).view(torch.int16)
+
+
 def stack_layer_device(layer: int, device, n_layers: int = 32, d_model: int = 4096, ffn: int = 14336,
                        outlier_rate: float = 1e-3, outlier_scale: float = 100.0):
-    """Layer `layer` of the 32-layer stack drawn on a torch device: the recipe
-    of `stack_layer` (the layer's sigma, N(0, sigma) weights, outliers at
-    `outlier_rate` scaled by `outlier_scale`, RNE to BF16) with torch's
-    generator seeded 2000 + 3*layer + j, so the values differ from
-    `stack_layer`'s.  Used where 96 full matrices must be made quickly (the
-    timed stack); returns three int16 tensors holding the BF16 patterns."""
-    import torch
+    """Layer `layer` of the 32-layer stack drawn on a torch device
+    (`weight_matrix_device` with the layer's sigma and seeds
+    2000 + 3*layer + j): gate, up, down as int16 tensors."""
     sigma = float(stack_sigmas(n_layers)[layer])
-    out = []
-    for j, (rows, cols) in enumerate(((ffn, d_model), (ffn, d_model), (d_model, ffn))):
-        g = torch.Generator(device=device)
-        g.manual_seed(2000 + 3 * layer + j)
-        w = torch.randn(rows, cols, generator=g, device=device, dtype=torch.float32) * sigma
-        if outlier_rate > 0:
-            mask = torch.rand(rows, cols, generator=g, device=device) < outlier_rate
-            w = torch.where(mask, w * outlier_scale, w)
-        out.append(w.to(torch.bfloat16).view(torch.int16))
-        del w
-    return tuple(out)
+    shapes = ((ffn, d_model), (ffn, d_model), (d_model, ffn))
+    return tuple(weight_matrix_device(r, c, sigma, outlier_rate, outlier_scale, 2000 + 3 * layer + j, device)
+                 for j, (r, c) in enumerate(shapes))
 
 
 def mlp_block(d_model: int = 4096, ffn: int = 14336, sigma: float = 0.02,
