@@ -39,9 +39,9 @@ HBM_FALLBACK_GBS = 6650.0
 # of the direct-palette GEMM kernel (the 14336x4096 gate projection at batch 8,
 # from one ncu --set full capture), valid only for the kernel sources it was
 # taken on: reported as null once they change.
-NCU_TRAFFIC = {"bytes_per_launch": 93671936,
+NCU_TRAFFIC = {"bytes_per_launch": 93159936,
                "launch": "gate projection 14336x4096, batch 8",
-               "sources_sha256": "682f3dec5e0ee4221e4987950b3c2ec2811d32554a1ddb771f7f3e7d7578910d"}
+               "sources_sha256": "fe60dd15088e342568183b6c5cd62478789e0968dc1475fd6c50d1ac6731f3b1"}
 GEMM_SOURCES = ["mlp_huffman_coded_b200/csrc/uw_gemm.cu", "mlp_huffman_coded_b200/csrc/uw_device.cuh",
                 "mlp_huffman_coded_b200/csrc/uw_internal.h"]
 
@@ -362,7 +362,32 @@ def run_gpu(args, world, rank, local):
 
     per_step_bytes = step_bytes(B)
     t_step = ms / 1e3 / args.steps
-    achieved = per_step_bytes / t_step / 1e9
+    # a step is 3 launches of the GEMM kernel back to back (gate, up with the
+    # fused SwiGLU, down); they tile the step, so the average launch lasts a
+    # third of it and moves a third of its algorithmic bytes
+    launch_s = t_step / 3
+    bytes_per_launch = per_step_bytes / 3
+    achieved = bytes_per_launch / launch_s / 1e9
+
+    # the gate launch alone, timed launch by launch with CUDA events on the
+    # launching stream, L2 flushed before each (outside the timed interval)
+    flush = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+    ws_g = uw.Workspace(uw.workspace_bytes(dms[0], uw.PIPE_DIRECT, B), device=dev)
+    g_out = torch.empty(B, FFN, dtype=torch.int16, device=dev)
+    iso = []
+    for i in range(args.warmup + 20):
+        flush.view(torch.int32).max()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        uw.gemm_direct_palette(dms[0], x, g_out, ws_g, stream)
+        a1.record(stream)
+        a1.synchronize()
+        if i >= args.warmup:
+            iso.append(a0.elapsed_time(a1) / 1e3)
+    ws_g.check("gate launch")
+    iso_s = float(np.median(iso))
+    gate_bytes = dms[0].direct_palette_bytes() + 2 * B * (D_MODEL + FFN)
+    del ws_g, g_out, flush
 
     # the other batches the block is quoted at (1 and 32 next to the default
     # 8): the same step, timed the same way, plus the BF16 comparator
@@ -425,9 +450,16 @@ def run_gpu(args, world, rank, local):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": ncu_traffic_per_launch(),
                          "traffic_launch": NCU_TRAFFIC["launch"],
-                         "kernel": "gemm_kernel<PACK, uniform palette> (direct palette; 3 launches per step, "
-                                   "achieved = algorithmic bytes per step / step time)",
-                         "algorithmic_bytes_per_step": per_step_bytes, "peak_source": f"{src} hbm_gbs"},
+                         "kernel": "gemm_kernel<PACK, uniform palette> (direct-palette reconstructive GEMM)",
+                         "launches_per_step": 3, "avg_launch_us": launch_s * 1e6,
+                         "algorithmic_bytes_per_launch": bytes_per_launch,
+                         "algorithmic_bytes_per_step": per_step_bytes,
+                         "isolated_gate_launch": {"us": iso_s * 1e6, "algorithmic_bytes": gate_bytes,
+                                                  "achieved_gbs": gate_bytes / iso_s / 1e9,
+                                                  "frac": gate_bytes / iso_s / 1e9 / peak,
+                                                  "timing": "median of 20 launches, CUDA events on the launching "
+                                                            "stream, L2 flushed before each"},
+                         "peak_source": f"{src} hbm_gbs ({'of measured' if src == 'measured' else 'of fallback'})"},
             "effective_weight_gbs": weight_gbs,
             "other_batches": other,
             "bf16_torch_matmul_ms_per_step": bf16_ms,
