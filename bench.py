@@ -41,7 +41,7 @@ HBM_FALLBACK_GBS = 6650.0
 # taken on: reported as null once they change.
 NCU_TRAFFIC = {"bytes_per_launch": 93159936,
                "launch": "gate projection 14336x4096, batch 8",
-               "sources_sha256": "fe60dd15088e342568183b6c5cd62478789e0968dc1475fd6c50d1ac6731f3b1"}
+               "sources_sha256": "628df866d5af27fe50260c8255cf485bfb5872de899c62137d64b8f486b81cf9"}
 GEMM_SOURCES = ["mlp_huffman_coded_b200/csrc/uw_gemm.cu", "mlp_huffman_coded_b200/csrc/uw_device.cuh",
                 "mlp_huffman_coded_b200/csrc/uw_internal.h"]
 

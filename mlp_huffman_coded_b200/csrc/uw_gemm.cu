@@ -28,10 +28,12 @@
 //    The producer is one thread running a short loop; the weight copies of
 //    the first stages leave before any table is read.
 //  * Persistent CTAs, one per SM, split the linearised (tile, k-block) space
-//    evenly (stream-K); a tile split across CTAs is finished by its first
-//    contributor, which adds the others' published partial sums to its own
-//    (still in TMEM) in CTA order, so the result does not depend on timing
-//    and is identical for every pipeline and stage size.
+//    evenly (stream-K); every contributor to a tile split across CTAs writes
+//    its partial sums to its own slot and takes a ticket, and the last to
+//    arrive adds all the slots in CTA order and stores y, so nobody waits for
+//    another CTA and the result does not depend on timing: it is identical
+//    for every pipeline and stage size.  The tile counters sit in a fixed
+//    region of the workspace and are back at zero after every launch.
 //  * FP32 accumulators live in TMEM; the epilogue reads them with tcgen05.ld,
 //    rounds to nearest-even BF16 (optionally applying SiLU(g) * u) and writes
 //    16-row chunks through shared memory with TMA tensor stores.
