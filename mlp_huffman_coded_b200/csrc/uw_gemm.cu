@@ -124,6 +124,7 @@ struct KParams {
   int n_soff;         // its capacity in words
   uint32_t a_col0;    // first TMEM column of the rebuilt A tiles (32 per k-block)
   uint32_t epi_off;   // epilogue staging: 2 output chunks (+ 2 gate chunks)
+  uint32_t ring_bytes;  // shared memory of the weight and activation rings (from 0)
   int tma_out;        // outputs leave through TMA tensor stores (else per element)
   int x3d;            // a stage's activation tiles arrive in one 3-D TMA load
 };
@@ -137,6 +138,7 @@ struct Bars {
   uint64_t acc_full[2], acc_empty[2], drain[kMaxIssuers];
   uint64_t meta_full[2];
   uint64_t gate_full[2];  // fused SwiGLU: gate chunk landed
+  uint64_t part_full;     // split-K: the other contributors' partial sums landed in the rings
   uint32_t tmem_base;
   uint32_t abort;
   uint32_t last_arriver;  // epilogue: this CTA completed a split tile
@@ -436,6 +438,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         mbar_init(&bars->gate_full[i], 1);
       }
       for (int i = 0; i < kMaxIssuers; ++i) mbar_init(&bars->drain[i], 1);
+      mbar_init(&bars->part_full, 1);
       bars->abort = 0;
       mbar_fence_init();
       if constexpr (!kIdx4) {
@@ -914,15 +917,21 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         // arrive adds all partials in CTA order and stores y.  Nobody waits
         // for another CTA, and the sum is the same whoever finishes last.
         const int64_t slot0 = t + c_first;
-        float* my_part = p.partials + ((slot0 + (blockIdx.x - c_first)) * 128 + r) * p.ntile;
+        // a contributor's part: its slot of 128 x ntile sums, chunk-major
+        // ([chunk][row][16 columns]) so each chunk is 8 KB in one piece
+        const int64_t slot_floats = 128 * static_cast<int64_t>(p.ntile);
+        float* my_part = p.partials + (slot0 + (blockIdx.x - c_first)) * slot_floats + r * 16;
         for (int cc = 0; cc < n_chunks; ++cc) {
           float acc[16];
           own_sum(cc, acc);
-          float4* dst = reinterpret_cast<float4*>(my_part + cc * 16);
+          float4* dst = reinterpret_cast<float4*>(my_part + cc * (128 * 16));
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4)
             dst[q4] = make_float4(acc[4 * q4], acc[4 * q4 + 1], acc[4 * q4 + 2], acc[4 * q4 + 3]);
         }
+        // the partial sums may be read by another CTA's bulk copy (or this
+        // one's): order the stores before asynchronous-proxy reads
+        fence_proxy_async_global();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->acc_empty[ab]);
@@ -936,14 +945,63 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         group_sync();  // the flag, and the acquired partials, for the whole group
         if (*last_flag) {
           if (tma_gate && elected && n_chunks > 0) load_gate(ch, mt, b_first);
-          for (int cc = 0; cc < n_chunks && ok; ++cc) {
+          // The CTA's last segment: its rings are idle (every stage has been
+          // rebuilt and multiplied), so the parts come into them by bulk
+          // copies, as many chunks of every contributor at a time as fit (one
+          // round trip per batch of chunks); otherwise each chunk's parts are
+          // read from L2 one after the other.  Either way the sum is every
+          // part, in CTA order.
+          constexpr uint32_t kChunkPart = 128u * 16u * 4u;  // one contributor's chunk
+          const uint32_t fit = p.ring_bytes / (static_cast<uint32_t>(ncontrib) * kChunkPart);
+          const int per_batch = static_cast<int>(min(static_cast<uint32_t>(n_chunks), fit));
+          const bool staged = seg_end >= u1 && per_batch >= 1;
+          const int64_t slot_floats = 128 * static_cast<int64_t>(p.ntile);
+          uint32_t batch_no = 0;
+          for (int cb = 0; cb < n_chunks && ok; cb += staged ? per_batch : n_chunks) {
+          const int nb = staged ? min(per_batch, n_chunks - cb) : n_chunks;
+          if (staged) {
+            // the previous batch has been read out of shared memory
+            group_sync();
+            if (elected) {
+              // the parts were published to this thread (acquire): order
+              // that, and the reads of the previous batch, before the
+              // asynchronous-proxy copies
+              fence_proxy_async_global();
+              fence_proxy_async_smem();
+              mbar_arrive_expect_tx(&bars->part_full, static_cast<uint32_t>(ncontrib * nb) * kChunkPart);
+              for (int jc = 0; jc < ncontrib; ++jc)
+                bulk_load(smem + static_cast<size_t>(jc) * per_batch * kChunkPart,
+                          p.partials + (slot0 + jc) * slot_floats + static_cast<int64_t>(cb) * (128 * 16),
+                          static_cast<uint32_t>(nb) * kChunkPart, &bars->part_full);
+            }
+            ok = mbar_wait(&bars->part_full, batch_no & 1, &bars->abort, p.status);
+            ok = group_and(__all_sync(0xFFFFFFFFu, ok));
+            ++batch_no;
+            if (!ok) {
+              // the copies must land before the shared memory goes away
+              if (elected) mbar_wait(&bars->part_full, (batch_no - 1) & 1, nullptr, p.status);
+              break;
+            }
+          }
+          for (int cc = cb; cc < cb + nb && ok; ++cc) {
             float acc[16];
             for (int jc = 0; jc < ncontrib; ++jc) {
-              const float4* src =
-                  reinterpret_cast<const float4*>(p.partials + ((slot0 + jc) * 128 + r) * p.ntile + cc * 16);
               float4 w4[4];
+              if (staged) {
+                const uint32_t a = smem_s + (static_cast<uint32_t>(jc * per_batch + (cc - cb)) * 128u +
+                                             static_cast<uint32_t>(r)) * 64u;
 #pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) w4[q4] = __ldcg(src + q4);
+                for (int q4 = 0; q4 < 4; ++q4) {
+                  const uint4 u4 = lds128(a + q4 * 16);
+                  w4[q4] = make_float4(__uint_as_float(u4.x), __uint_as_float(u4.y), __uint_as_float(u4.z),
+                                       __uint_as_float(u4.w));
+                }
+              } else {
+                const float4* src = reinterpret_cast<const float4*>(
+                    p.partials + (slot0 + jc) * slot_floats + (static_cast<int64_t>(cc) * 128 + r) * 16);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) w4[q4] = __ldcg(src + q4);
+              }
 #pragma unroll
               for (int q4 = 0; q4 < 4; ++q4) {
                 acc[4 * q4] = jc ? acc[4 * q4] + w4[q4].x : w4[q4].x;
@@ -958,6 +1016,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             }
             if (tma_gate && elected && cc + 1 < n_chunks) load_gate(ch, mt, b_first + (cc + 1) * 16);
           }
+          }  // chunk batches
           if (!ok) break;
         }
         group_sync();  // the flag word is reused by the next split segment
@@ -1299,6 +1358,7 @@ uw_status launch_gemm(const GemmArgs& a, cudaStream_t s) {
   kp.n_soff = lay.n_soff;
   kp.a_col0 = lay.a_col0;
   kp.epi_off = lay.epi_off;
+  kp.ring_bytes = lay.ring_bytes;
   kp.tma_out = tma_out ? 1 : 0;
   kp.x3d = x3d;
 
