@@ -343,7 +343,7 @@ UW_API uw_status uw_decode_exponent_only(const uw_matrix* m, uint8_t* out_exp8, 
  * [n_rows, cols] (device) row i = row rows[i] of W, bit for bit.  rows:
  * device int32[n_rows]; repeats allowed.  Only the chunks that hold a
  * requested row are decoded.  Errors as uw_decode_full, plus
- * UW_ERR_INVALID_ARG for n_rows < 0 or NULL rows; a row id outside
+ * UW_ERR_INVALID_ARG for n_rows < 0 or NULL / misaligned rows; a row id outside
  * [0, rows) is found on the device: that output row is zeros and the
  * status word records UW_ERR_INVALID_ARG. */
 UW_API uw_status uw_decode_rows(const uw_matrix* m, const int32_t* rows, int32_t n_rows, uint16_t* out_bf16,

@@ -531,7 +531,7 @@ uw_status launch_decode(const uw_matrix* m, int mode, void* out, uint32_t* statu
 
 uw_status launch_decode_rows(const uw_matrix* m, const int32_t* rows, int64_t n_rows, void* out, uint32_t* status,
                              cudaStream_t s) {
-  if (n_rows < 0 || (n_rows > 0 && !rows)) return UW_ERR_INVALID_ARG;
+  if (n_rows < 0 || (n_rows > 0 && (!rows || reinterpret_cast<uintptr_t>(rows) % 4 != 0))) return UW_ERR_INVALID_ARG;
   DecodeParams p;
   uw_status st = fill_params(m, out, status, &p);
   if (st != UW_OK) return st;

@@ -212,3 +212,19 @@ def test_decode_rows_outside_the_matrix_are_reported():
     assert e.value.status == uw.UW_ERR_INVALID_ARG
     assert np.array_equal(got[0], w[3]) and np.array_equal(got[3], w[99])
     assert not got[1].any() and not got[2].any()
+
+
+def test_decode_rows_argument_errors():
+    """Rejected on the host before anything is launched: a negative count
+    and a row-id pointer that is not 4-byte aligned."""
+    import ctypes as C
+    import torch
+    w = synth.weight_matrix(64, 256, 0.02, 0.0, 1.0, 106)
+    dm = device_matrix(w, direct=False)
+    ws = uw.Workspace(256)
+    ids = torch.zeros(8, dtype=torch.int32, device="cuda")
+    out = empty_bf16(4, 256)
+    f = uw.lib().uw_decode_rows
+    assert f(C.byref(dm.mat), ids.data_ptr(), -1, out.data_ptr(), ws.ptr, ws.nbytes, None) == uw.UW_ERR_INVALID_ARG
+    assert f(C.byref(dm.mat), ids.data_ptr() + 2, 4, out.data_ptr(), ws.ptr, ws.nbytes, None) == uw.UW_ERR_INVALID_ARG
+    ws.check("no launch happened")
