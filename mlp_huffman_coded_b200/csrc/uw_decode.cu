@@ -10,23 +10,27 @@
 //
 // Work split.  The stream is cut into chunks of `chunk_groups` 64-element
 // groups, each with its own start bit.  A warp takes 32 consecutive chunks
-// (one per lane) in two steps:
-//   1. each lane decodes its chunk's coded groups into 4-bit palette indices:
-//      a 32-bit window over three prefetched stream words (funnel shift), one
-//      shared-memory table lookup per 11 bits yielding every whole code in
-//      them (up to 4 indices, their total length and count), and the indices
-//      packed 8 to a word into the warp's shared-memory stage.  Codes longer
-//      than the table (the rare tail of the exponent distribution) take the
-//      canonical first-code comparison.  This step is the same whatever the
-//      output format;
-//   2. the warp writes the 32 chunks' groups together: consecutive lanes take
+// (one per lane) in three steps:
+//   1. the warp copies the stream words its 32 chunks span (one contiguous
+//      range) into shared memory with coalesced loads;
+//   2. each lane decodes its chunk's coded groups into 4-bit palette indices:
+//      a 64-bit window over the staged words, refilled once per four table
+//      lookups; each lookup takes the window's top 11 bits and yields every
+//      whole code in them (up to 4 indices, their total length and count);
+//      the indices collect in a 64-bit register and go 8 to a word into the
+//      lane's region of the warp's shared-memory stage (coded groups in
+//      order, 8 words each; an odd region stride keeps the lanes' stores on
+//      distinct banks).  Codes longer than the table (the rare tail of the
+//      exponent distribution) take the canonical first-code comparison.
+//      This step is the same whatever the output format;
+//   3. the warp writes the 32 chunks' groups together: consecutive lanes take
 //      consecutive 16-byte pieces of the output, so every store (and, for the
 //      full decode, every sign+mantissa load) is coalesced.  Indices become
 //      exponent bytes by a byte-permute palette lookup; verbatim groups come
 //      from the verbatim store.
 // A chunk whose codes do not end exactly at the next chunk's offset, or an
 // invalid code, records UW_ERR_CORRUPT; every stream read stays inside the
-// stream and every verbatim read inside the store.
+// stream (or the staged copy) and every verbatim read inside the store.
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -43,11 +47,14 @@ namespace {
 
 constexpr int kLutBits = 11;
 constexpr int kLutSize = 1 << kLutBits;
-constexpr int kStageBudget = 48 * 1024;  // per block: index stage + group info
-// Row gather: each warp first copies the stream words of its chunks into
-// shared memory with coalesced loads (a few warps decode a few rows, so the
-// lanes' dependent refills would otherwise each wait for HBM).
-constexpr int kRowStreamWords = 2048;
+// Dynamic shared memory per block (stage, group info and staged stream of
+// every warp): one block per SM shares one copy of the tables.  With
+// 4-group chunks a warp takes ~8 KB, so 25 warps fit; 25 x 32 threads leave
+// 80 registers a thread.
+constexpr int kBlockSmem = 200 * 1024;
+constexpr int kMaxWarps = 25;
+// Full decode: sign+mantissa loads in flight per lane in the write step.
+constexpr int kEmitBatch = 8;
 
 enum DecodeMode { kFull = 0, kExp8 = 1, kIdx4 = 2 };
 
@@ -69,6 +76,7 @@ struct DecodeParams {
   int64_t n_items;          // warp work items: 32-chunk batches (of each gathered row)
   int32_t batches_per_row;  // row gather
   int32_t chunk_groups;
+  uint32_t cg_magic;  // ceil(2^16 / chunk_groups): i / chunk_groups = (i * cg_magic) >> 16 for i <= 512
   int32_t gpr;  // groups per row
   int32_t wpr;  // flag words per row
   int32_t max_len;
@@ -77,16 +85,33 @@ struct DecodeParams {
   uint8_t code_len[16];
 };
 
+// Table entry: the whole codes at the head of the window, as
+//   bits 0..3  their total length (bits 4..6 zero, so a funnel shift can
+//              take the entry as its shift amount and four lengths add up
+//              in the low 6 bits),
+//   bit 7      kLong: the first code is longer than the table (the entry is
+//              kLong alone: it consumes and yields nothing),
+//   bits 8..23 their palette indices, 4 bits each, first code lowest,
+//   bits 27..31 4 x their count.
+constexpr uint32_t kLong = 0x80u;
+__host__ __device__ constexpr uint32_t entry(uint32_t len, uint32_t idx, uint32_t count) {
+  return len | (idx << 8) | ((4u * count) << 27);
+}
+
 struct DecodeTables {
-  // Every whole code inside each 11-bit prefix (at most 4): x = their
-  // palette indices (4 bits each, first code lowest) | cumulative lengths
-  // after 1..4 codes (4 bits each) << 16; y = count | total length << 8
-  // (count 0: the first code is longer than the table).
-  uint2 multi[kLutSize];
-  uint32_t first[17];   // first canonical code of each length
-  uint32_t count[17];   // codes of each length
-  uint32_t offset[17];  // index of the first symbol of each length
-  uint8_t sorted[16];   // symbols in (length, index) order
+  // Every whole code inside each 11-bit prefix (at most 4), or kLong.
+  uint32_t multi[kLutSize];
+  uint16_t cum[kLutSize];  // lengths after 1..4 of those codes, 4 bits each
+  // Codes longer than the table: canonical codes put their 11-bit prefixes
+  // in one range from long_base up, at most 15 of them (16 symbols).  Row r
+  // (prefix long_base + r) holds the code of each value of the next 4 bits,
+  // as a one-code entry; row 16 and unmatched bits are 0 (invalid).
+  uint32_t sub[17 * 16];
+  uint32_t long_base;
+  uint32_t first[17];      // first canonical code of each length
+  uint32_t count[17];      // codes of each length
+  uint32_t offset[17];     // index of the first symbol of each length
+  uint8_t sorted[16];      // symbols in (length, index) order
 };
 
 // lut: kLutSize words of scratch (the first code of each prefix, sym |
@@ -135,6 +160,23 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables
     lut[v] = ent;
   }
   __syncthreads();
+  {
+    const uint32_t base = t.first[kLutBits] + t.count[kLutBits];  // end of the codes of <= 11 bits
+    if (threadIdx.x == 0) t.long_base = base;
+    for (int s = threadIdx.x; s < 17 * 16; s += blockDim.x) {
+      const uint32_t row = static_cast<uint32_t>(s) >> 4;
+      const uint32_t val = ((base + row) << 4) | (static_cast<uint32_t>(s) & 15u);  // 15-bit value
+      uint32_t ent = 0;
+      for (int l = kLutBits + 1; row < 16 && l <= p.max_len; ++l) {
+        const uint32_t d = (val >> (15 - l)) - t.first[l];
+        if (t.count[l] && d < t.count[l]) {
+          ent = entry(static_cast<uint32_t>(l), t.sorted[t.offset[l] + d], 1);
+          break;
+        }
+      }
+      t.sub[s] = ent;
+    }
+  }
   // chain single-code lookups inside the 11-bit prefix: a code shorter than
   // the bits left is decoded correctly whatever the zero padding (prefix-free)
   for (int v = threadIdx.x; v < kLutSize; v += blockDim.x) {
@@ -149,46 +191,48 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables
       cum |= static_cast<uint32_t>(used) << (4 * n);
       ++n;
     }
-    t.multi[v] = make_uint2(idx | (cum << 16), static_cast<uint32_t>(n) | (static_cast<uint32_t>(used) << 8));
+    t.multi[v] = n ? entry(static_cast<uint32_t>(used), idx, static_cast<uint32_t>(n)) : kLong;
+    t.cum[v] = static_cast<uint16_t>(cum);
   }
   __syncthreads();
 }
 
-// A code longer than the table by canonical first-code comparison over the
-// left-aligned 32-bit window: symbol | length << 4.  An invalid code records
-// UW_ERR_CORRUPT and reads as symbol 0 of length 1, so decoding stays bounded.
-__device__ __noinline__ uint32_t decode_long(const DecodeTables& t, int max_len, uint32_t* status, uint32_t win) {
-  for (int l = kLutBits + 1; l <= max_len; ++l) {
-    const uint32_t d = (win >> (32 - l)) - t.first[l];
-    if (t.count[l] && d < t.count[l]) return t.sorted[t.offset[l] + d] | (static_cast<uint32_t>(l) << 4);
+// The code at a prefix v whose first code is longer than the table, from
+// the second-level rows (win: the left-aligned window).  An invalid code
+// records UW_ERR_CORRUPT and reads as symbol 0 of length 1, so decoding stays
+// bounded.
+__device__ __forceinline__ uint32_t long_code(const DecodeTables& t, uint32_t* status, uint32_t v, uint32_t win) {
+  const uint32_t row = min(v - t.long_base, 16u);  // wraps below the range, then clamps to the invalid row
+  uint32_t e = t.sub[row * 16 + ((win >> (32 - 15)) & 15u)];
+  if (e == 0) {
+    record_status(status, UW_ERR_CORRUPT);
+    e = entry(1, 0, 1);
   }
-  record_status(status, UW_ERR_CORRUPT);
-  return 1u << 4;
+  return e;
 }
 
-// Word w of a lane's stage region (8 words per chunk group): 4-word units
-// XOR-swizzled by the lane so lanes writing the same word mostly hit
-// different banks; a unit stays contiguous (16-byte reads).  umask + 1 is a
-// power of two dividing the region's unit count, so the swizzle stays inside
-// the region.
-__device__ __forceinline__ uint32_t stage_word(int lane, int w, int cg, int umask) {
-  return static_cast<uint32_t>(lane * 8 * cg + (((w >> 2) ^ (lane & umask)) << 2) + (w & 3));
+// Bulk prefetch of [src, src + bytes) into L2 (16-byte multiples; a hint
+// that nothing waits for).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+               : "memory");
 }
 
-// Step 1: the lane decodes chunk c into its stage region (coded groups at
-// their slots, 8 words each) and records every group's source in info[]:
-// -1 coded, >= 0 verbatim slot, -2 unreadable verbatim slot (written as
-// zeros), -3 past the matrix.
-// sbuf (may be NULL): stream words [sbase, sbase + sn) in shared memory.
-__device__ __forceinline__ void decode_chunk(const DecodeParams& p, const DecodeTables& t, int64_t c, int lane,
-                                             uint32_t* stage, int32_t* info, int umask, const uint32_t* sbuf,
-                                             int64_t sbase, int64_t sn) {
+// Info word of a coded group: -16 - (its rank among the chunk's coded
+// groups); the rank places it in the lane's stage region.
+constexpr int32_t kCodedBase = -16;
+
+// The sources of chunk c's groups into inf[s]: kCodedBase - rank for a
+// coded group (its rank among the chunk's coded groups places it in the
+// lane's stage region), >= 0 verbatim slot, -2 unreadable verbatim slot
+// (written as zeros), -3 past the matrix.  Returns the coded groups.
+__device__ __forceinline__ int group_sources(const DecodeParams& p, int64_t c, int32_t* inf) {
   const int cg = p.chunk_groups;
   const int64_t g0 = c * cg;
   const int64_t g1 = min(g0 + cg, p.n_groups);
   int64_t r = g0 / p.gpr;
   int32_t j = static_cast<int32_t>(g0 - r * p.gpr);
-  uint32_t coded = 0;
+  int n_coded = 0;
   for (int s = 0; s < cg; ++s) {
     int32_t v = -3;
     if (g0 + s < g1) {
@@ -204,106 +248,121 @@ __device__ __forceinline__ void decode_chunk(const DecodeParams& p, const Decode
           v = -2;
         }
       } else {
-        v = -1;
-        coded |= 1u << s;
+        v = kCodedBase - n_coded;
+        ++n_coded;
       }
       if (++j == p.gpr) {
         j = 0;
         ++r;
       }
     }
-    info[lane * cg + s] = v;
+    inf[s] = v;
   }
-  const uint32_t b0 = __ldg(p.off + c), b1 = __ldg(p.off + c + 1);
-  const int64_t last_word = p.stream_words - 1;
-  auto fetch = [&](int64_t i) -> uint32_t {
-    const int64_t k = i - sbase;
-    return (sbuf && k >= 0 && k < sn) ? sbuf[k] : __ldg(p.stream + min(i, last_word));
-  };
-  int64_t wi = b0 >> 5;
-  uint32_t w0 = fetch(wi);
-  uint32_t w1 = fetch(wi + 1);
-  uint32_t w2 = fetch(wi + 2);
-  wi += 3;
-  int bp = static_cast<int>(b0 & 31);
-  uint32_t consumed = 0;
-  const int total = 64 * __popc(coded);
-  int done = 0;
-  uint32_t acc_lo = 0, acc_hi = 0;  // pending indices, first lowest
-  int nacc = 0;                     // indices pending (< 8 between steps)
-  uint32_t left = coded;            // coded groups not started yet
-  int slot = 0, wq = 8;             // current group's slot, words written into it
-  // Both steps are written to compile to selects and predicated memory
-  // operations rather than branches: lanes of a warp flush and refill at
-  // different times.
-  auto push = [&](uint32_t idx, int cnt) {
-    const int sh = 4 * nacc;
-    const uint64_t a = (static_cast<uint64_t>(acc_hi) << 32 | acc_lo) | (static_cast<uint64_t>(idx) << sh);
-    nacc += cnt;
-    const bool full = nacc >= 8;  // 8 indices -> the stage
-    const bool start = full && wq == 8;
-    slot = start ? __ffs(left) - 1 : slot;
-    left = start ? left & (left - 1) : left;
-    wq = start ? 0 : wq;
-    if (full) stage[stage_word(lane, slot * 8 + wq, cg, umask)] = static_cast<uint32_t>(a);
-    wq += full ? 1 : 0;
-    acc_lo = full ? static_cast<uint32_t>(a >> 32) : static_cast<uint32_t>(a);
-    acc_hi = full ? 0u : static_cast<uint32_t>(a >> 32);
-    nacc -= full ? 8 : 0;
-  };
-  auto advance = [&](int len) {
-    bp += len;
-    consumed += static_cast<uint32_t>(len);
-    const bool cross = bp >= 32;
-    uint32_t nw = 0;
-    if (cross) nw = fetch(wi);
-    bp -= cross ? 32 : 0;
-    w0 = cross ? w1 : w0;
-    w1 = cross ? w2 : w1;
-    w2 = cross ? nw : w2;
-    wi += cross ? 1 : 0;
-  };
-  // whole lookups while at least 4 indices remain (two per check)
-  auto step = [&]() {
-    const uint32_t win = __funnelshift_l(w1, w0, bp);
-    const uint2 e = t.multi[win >> (32 - kLutBits)];
-    int cnt = static_cast<int>(e.y & 7);
-    uint32_t idx = e.x & 0xFFFFu;
-    int len = static_cast<int>(e.y >> 8);
-    if (cnt == 0) {
-      const uint32_t d = decode_long(t, p.max_len, p.status, win);
-      idx = d & 15u;
-      len = static_cast<int>(d >> 4);
-      cnt = 1;
-    }
-    push(idx, cnt);
-    advance(len);
-    done += cnt;
-  };
-  while (total - done >= 8) {
-    step();
-    step();
-  }
-  while (total - done >= 4) step();
-  // the last indices one code at a time
-  while (done < total) {
-    const uint32_t win = __funnelshift_l(w1, w0, bp);
-    const uint2 e = t.multi[win >> (32 - kLutBits)];
-    uint32_t idx;
-    int len;
-    if ((e.y & 7) == 0) {
-      const uint32_t d = decode_long(t, p.max_len, p.status, win);
-      idx = d & 15u;
-      len = static_cast<int>(d >> 4);
+  return n_coded;
+}
+
+// Step 2: the lane decodes the n_coded coded groups of a chunk whose codes
+// span bits [b0, b1) into st[8 * rank ...].  SMEM: stream words [sbase,
+// sbase + smax + 3) are staged in sb (reads clamp into it); else they come
+// from global memory.
+template <bool SMEM>
+__device__ __forceinline__ void decode_chunk(const DecodeParams& p, const DecodeTables& t, uint32_t b0, uint32_t b1,
+                                             int n_coded, uint32_t* st, const uint32_t* sb, uint32_t sbase,
+                                             uint32_t smax) {
+  const uint32_t last_word = static_cast<uint32_t>(p.stream_words - 1);
+  // window: bits [pos, pos + 64) of the stream, left-aligned in hi:lo; SMEM
+  // keeps pos relative to the staged copy
+  uint32_t pos = SMEM ? b0 - (sbase << 5) : b0, hi = 0, lo = 0;
+  auto refill = [&]() {
+    const uint32_t wi = pos >> 5;
+    uint32_t a, b, d;
+    if (SMEM) {
+      const uint32_t k = min(wi, smax);  // a corrupt offset clamps into the copy
+      a = sb[k];
+      b = sb[k + 1];
+      d = sb[k + 2];
     } else {
-      idx = e.x & 15u;
-      len = static_cast<int>((e.x >> 16) & 15);
+      a = __ldg(p.stream + min(wi, last_word));
+      b = __ldg(p.stream + min(wi + 1, last_word));
+      d = __ldg(p.stream + min(wi + 2, last_word));
     }
-    push(idx, 1);
-    advance(len);
-    ++done;
+    hi = __funnelshift_l(b, a, pos);  // shift by pos mod 32
+    lo = __funnelshift_l(d, b, pos);
+  };
+  uint64_t acc = 0;  // pending indices, first lowest
+  uint32_t nsh = 0;  // their bits (4 per index)
+  uint32_t wq = 0;   // stage words written
+  const uint32_t total4 = 256u * static_cast<uint32_t>(n_coded);  // 4 x indices to decode
+  // Consume an entry's codes: the window moves by its length (the entry's
+  // low 5 bits), its indices go into acc.
+  auto take = [&](uint32_t e) {
+    hi = __funnelshift_l(lo, hi, e);
+    lo = __funnelshift_l(0u, lo, e);
+    acc |= static_cast<uint64_t>(__byte_perm(e, 0, 0x4421)) << nsh;
+    nsh += e >> 27;
+  };
+  auto look = [&]() {
+    const uint32_t e = t.multi[hi >> (32 - kLutBits)];
+    take(e);
+    return e;
+  };
+  // a whole word of indices -> the stage (a select, not a branch: lanes
+  // fill words at different times)
+  auto flush = [&]() {
+    const bool f = nsh >= 32;
+    if (f) st[wq] = static_cast<uint32_t>(acc);
+    acc = f ? (acc >> 32) : acc;
+    wq += f ? 1u : 0u;
+    nsh -= f ? 32u : 0u;
+  };
+  // one code longer than the table at the head of the window
+  auto long_step = [&]() {
+    const uint32_t e = long_code(t, p.status, hi >> (32 - kLutBits), hi);
+    take(e);
+    pos += e & 15u;
+    flush();
+  };
+  refill();
+  // Four lookups per refill while at least 16 indices are left: a refill
+  // leaves 64 valid bits, four lookups take at most 44 and a long code 15
+  // more.  A long code stops the lookups at its position (kLong consumes
+  // nothing), so the fourth entry says whether one is waiting.
+  while (32u * wq + nsh + 64u <= total4) {
+    const uint32_t e1 = look();
+    const uint32_t e2 = look();
+    flush();
+    const uint32_t e3 = look();
+    const uint32_t e4 = look();
+    flush();
+    pos += (e1 + e2 + e3 + e4) & 63u;
+    if (e4 & kLong) long_step();
+    refill();
   }
-  if (consumed != b1 - b0) record_status(p.status, UW_ERR_CORRUPT);
+  while (32u * wq + nsh + 16u <= total4) {
+    const uint32_t e = look();
+    pos += e & 15u;
+    flush();
+    if (e & kLong) long_step();
+    refill();
+  }
+  while (32u * wq + nsh < total4) {
+    // the last indices: a lookup may hold more codes than the chunk has left
+    const uint32_t left4 = total4 - (32u * wq + nsh);
+    const uint32_t v = hi >> (32 - kLutBits);
+    uint32_t e = t.multi[v];
+    if (e & kLong) {
+      e = long_code(t, p.status, v, hi);
+    } else if ((e >> 27) > left4) {
+      const uint32_t n = left4 >> 2;
+      const uint32_t len = (static_cast<uint32_t>(t.cum[v]) >> (4 * (n - 1))) & 15u;
+      e = entry(len, (e >> 8) & ((1u << left4) - 1u), n);
+    }
+    take(e);
+    pos += e & 15u;
+    flush();
+    refill();
+  }
+  if (pos != (SMEM ? b1 - (sbase << 5) : b1)) record_status(p.status, UW_ERR_CORRUPT);
 }
 
 __device__ __forceinline__ uint32_t lookup4(const DecodeParams& p, uint32_t nib) {
@@ -325,63 +384,96 @@ __device__ __forceinline__ uint4 exponents16(const uint4& a, const uint4& b) {
   return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-// Step 2: the output pieces of batch groups [gl0, gl1) (batch group gi is
+// Words per lane stage region: 8 per chunk group, plus one so that lanes
+// storing their regions' same word hit distinct banks.
+__device__ __forceinline__ int region_words(int cg) { return 8 * cg + 1; }
+
+// Step 3: the output pieces of batch groups [gl0, gl1) (batch group gi is
 // slot gi % cg of lane gi / cg's chunk; matrix group g_batch0 + gi); og0 is
-// the output group of batch group gl0.  `zero`: write zeros.
+// the output group of batch group gl0.  `zero`: write zeros.  Each lane
+// takes kEmitBatch pieces at a time and issues all their loads first.
 template <int MODE>
 __device__ __forceinline__ void emit_groups(const DecodeParams& p, const uint32_t* stage, const int32_t* info,
-                                            int umask, int64_t g_batch0, int gl0, int gl1, int64_t og0,
-                                            bool zero) {
+                                            int64_t g_batch0, int gl0, int gl1, int64_t og0, bool zero) {
   constexpr int kPieces = MODE == kIdx4 ? 2 : (MODE == kExp8 ? 4 : 8);  // 16-byte pieces per group
-  const int cg = p.chunk_groups;
+  const int rw = region_words(p.chunk_groups);
   const int lane = threadIdx.x & 31;
   const int n = (gl1 - gl0) * kPieces;
-  for (int pc = lane; pc < n; pc += 32) {
-    const int gi = gl0 + pc / kPieces;
-    const int q = pc % kPieces;
-    const int L = gi / cg, s = gi - L * cg;
-    const int32_t v = zero ? -2 : info[gi];
-    const int64_t og = og0 + (gi - gl0);
-    uint4 o = make_uint4(0, 0, 0, 0);
-    if (MODE == kIdx4) {
-      if (v == -1) o = *reinterpret_cast<const uint4*>(stage + stage_word(L, s * 8 + 4 * q, cg, umask));
-      reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + og * 32)[q] = o;
-    } else if (MODE == kExp8) {
-      if (v == -1) {
-        const uint2 nw = *reinterpret_cast<const uint2*>(stage + stage_word(L, s * 8 + 2 * q, cg, umask));
-        o = make_uint4(lookup4(p, nw.x), lookup4(p, nw.x >> 16), lookup4(p, nw.y), lookup4(p, nw.y >> 16));
-      } else if (v >= 0) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.verbatim + static_cast<int64_t>(v) * 64) + 2 * q;
-        o = exponents16(__ldg(src), __ldg(src + 1));
+  for (int base = 0; base < n; base += 32 * kEmitBatch) {
+    int32_t vv[kEmitBatch];
+    uint4 raw[kEmitBatch];  // full decode: sm bytes (.x, .y) or a verbatim piece
+#pragma unroll
+    for (int u = 0; u < kEmitBatch; ++u) {
+      const int pc = base + u * 32 + lane;
+      const int gi = gl0 + pc / kPieces;
+      const int q = pc % kPieces;
+      vv[u] = pc < n ? (zero ? -2 : info[gi]) : -3;
+      raw[u] = make_uint4(0, 0, 0, 0);
+      if (MODE == kFull) {
+        if (vv[u] <= kCodedBase) {
+          const uint2 smv = __ldg(reinterpret_cast<const uint2*>(p.sm + (g_batch0 + gi) * 64) + q);
+          raw[u].x = smv.x;
+          raw[u].y = smv.y;
+        } else if (vv[u] >= 0) {
+          raw[u] = __ldg(reinterpret_cast<const uint4*>(p.verbatim + static_cast<int64_t>(vv[u]) * 64) + q);
+        }
       }
-      reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + og * 64)[q] = o;
-    } else {
-      if (v == -1) {
-        const uint32_t nw = stage[stage_word(L, s * 8 + q, cg, umask)];
-        const uint2 smv = __ldg(reinterpret_cast<const uint2*>(p.sm + (g_batch0 + gi) * 64) + q);
-        rebuild4(smv.x, lookup4(p, nw), o.x, o.y);
-        rebuild4(smv.y, lookup4(p, nw >> 16), o.z, o.w);
-      } else if (v >= 0) {
-        o = __ldg(reinterpret_cast<const uint4*>(p.verbatim + static_cast<int64_t>(v) * 64) + q);
+    }
+#pragma unroll
+    for (int u = 0; u < kEmitBatch; ++u) {
+      const int pc = base + u * 32 + lane;
+      if (pc >= n) break;
+      const int gi = gl0 + pc / kPieces;
+      const int q = pc % kPieces;
+      const int32_t v = vv[u];
+      const int L = static_cast<int>((static_cast<uint32_t>(gi) * p.cg_magic) >> 16);
+      const int64_t og = og0 + (gi - gl0);
+      // a coded group's first stage word
+      const uint32_t* sw = stage + L * rw + 8 * max(kCodedBase - v, 0);
+      uint4 o = make_uint4(0, 0, 0, 0);
+      if (MODE == kIdx4) {
+        if (v <= kCodedBase) o = make_uint4(sw[4 * q], sw[4 * q + 1], sw[4 * q + 2], sw[4 * q + 3]);
+        reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + og * 32)[q] = o;
+      } else if (MODE == kExp8) {
+        if (v <= kCodedBase) {
+          const uint32_t n0 = sw[2 * q], n1 = sw[2 * q + 1];
+          o = make_uint4(lookup4(p, n0), lookup4(p, n0 >> 16), lookup4(p, n1), lookup4(p, n1 >> 16));
+        } else if (v >= 0) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.verbatim + static_cast<int64_t>(v) * 64) + 2 * q;
+          o = exponents16(__ldg(src), __ldg(src + 1));
+        }
+        reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.out) + og * 64)[q] = o;
+      } else {
+        if (v <= kCodedBase) {
+          const uint32_t nw = sw[q];
+          rebuild4(raw[u].x, lookup4(p, nw), o.x, o.y);
+          rebuild4(raw[u].y, lookup4(p, nw >> 16), o.z, o.w);
+        } else if (v >= 0) {
+          o = raw[u];
+        }
+        reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + og * 64)[q] = o;
       }
-      reinterpret_cast<uint4*>(static_cast<uint16_t*>(p.out) + og * 64)[q] = o;
     }
   }
 }
 
+// Shared-memory words of one warp: stage, group info, staged stream.
+__host__ __device__ __forceinline__ int stream_cap_words(int cg) { return 192 * cg + 64; }
+__host__ __device__ __forceinline__ int warp_words(int cg) { return 32 * (8 * cg + 1) + 32 * cg + stream_cap_words(cg); }
+
 template <int MODE, bool ROWS>
-__global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(32 * kMaxWarps, 1) decode_kernel(const DecodeParams p) {
   __shared__ DecodeTables t;
   extern __shared__ __align__(16) uint32_t dsm[];
   build_tables(p, t, reinterpret_cast<uint16_t*>(dsm));  // the stage holds the build scratch
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int W = blockDim.x >> 5;
   const int cg = p.chunk_groups;
-  uint32_t* stage = dsm + warp * (256 * cg);
-  int32_t* info = reinterpret_cast<int32_t*>(dsm + W * 256 * cg) + warp * 32 * cg;
-  uint32_t* sbuf = ROWS ? dsm + W * 288 * cg + warp * kRowStreamWords : nullptr;
-  const int units = 2 * cg;
-  const int umask = min(units & -units, 8) - 1;
+  uint32_t* stage = dsm + warp * warp_words(cg);
+  int32_t* info = reinterpret_cast<int32_t*>(stage + 32 * region_words(cg));
+  uint32_t* sbuf = reinterpret_cast<uint32_t*>(info + 32 * cg);
+  const int64_t cap = stream_cap_words(cg);
+  const uint32_t last_word = static_cast<uint32_t>(p.stream_words - 1);
   for (int64_t it = static_cast<int64_t>(blockIdx.x) * W + warp; it < p.n_items;
        it += static_cast<int64_t>(gridDim.x) * W) {
     int64_t c_first, c_end, g_lo, g_hi, og0;
@@ -411,20 +503,48 @@ __global__ void __launch_bounds__(256) decode_kernel(const DecodeParams p) {
       g_hi = min(c_end * cg, rg1);
       og0 = i * p.gpr + (g_lo - rg0);
     }
-    int64_t sbase = 0, sn = 0;
-    if (ROWS && !zero) {
-      // the stream words of chunks [c_first, c_end), plus the three-word
-      // window's overrun, into the warp's buffer
-      sbase = __ldg(p.off + c_first) >> 5;
-      sn = min(static_cast<int64_t>((__ldg(p.off + c_end) >> 5) + 3 - sbase), static_cast<int64_t>(kRowStreamWords));
-      const int64_t last_word = p.stream_words - 1;
-      for (int64_t k = lane; k < sn; k += 32) sbuf[k] = __ldg(p.stream + min(sbase + k, last_word));
-      __syncwarp();
-    }
     const int64_t c = c_first + lane;
-    if (c < c_end && !zero) decode_chunk(p, t, c, lane, stage, info, umask, sbuf, sbase, sn);
+    const int nc = static_cast<int>(c_end - c_first);
+    // the next item's stream span (its offsets, loaded now) goes to L2
+    // while this one decodes; a full decode also prefetches this item's
+    // sign+mantissa bytes for step 3
+    uint32_t nb = 0;
+    const int64_t it_next = it + static_cast<int64_t>(gridDim.x) * W;
+    if (!ROWS && it_next < p.n_items && lane < 2) nb = __ldg(p.off + min(it_next * 32 + lane * 32, p.n_chunks));
+    if (MODE == kFull && !zero && lane == 0)
+      bulk_prefetch_l2(p.sm + g_lo * 64, static_cast<uint32_t>(g_hi - g_lo) * 64u);
+    if (!zero) {
+      // the lane's chunk offsets (consecutive lanes, consecutive words) and
+      // group sources, then step 1: the stream words of chunks [c_first,
+      // c_end) plus the window's two-word overrun, when they fit the warp's
+      // buffer
+      uint32_t b0 = 0, b1 = 0;
+      int n_coded = 0;
+      if (c < c_end) {
+        b0 = __ldg(p.off + c);
+        b1 = __ldg(p.off + c + 1);
+        n_coded = group_sources(p, c, info + lane * cg);
+      }
+      const uint32_t blo = __shfl_sync(0xffffffffu, b0, 0), bhi = __shfl_sync(0xffffffffu, b1, nc - 1);
+      const uint32_t sbase = blo >> 5;
+      const int64_t span = static_cast<int64_t>(bhi >> 5) + 3 - sbase;
+      uint32_t* st = stage + lane * region_words(cg);
+      if (bhi >= blo && span <= cap) {
+        for (int64_t k = lane; k < span; k += 32) sbuf[k] = __ldg(p.stream + min(sbase + static_cast<uint32_t>(k), last_word));
+        __syncwarp();
+        if (c < c_end) decode_chunk<true>(p, t, b0, b1, n_coded, st, sbuf, sbase, static_cast<uint32_t>(span - 3));
+      } else if (c < c_end) {
+        decode_chunk<false>(p, t, b0, b1, n_coded, st, nullptr, 0, 0);
+      }
+    }
+    if (!ROWS && it_next < p.n_items) {
+      const uint32_t nlo = __shfl_sync(0xffffffffu, nb, 0), nhi = __shfl_sync(0xffffffffu, nb, 1);
+      const uint32_t w0 = (nlo >> 5) & ~3u;
+      const uint32_t w1 = min(((nhi >> 5) + 6u) & ~3u, static_cast<uint32_t>(p.stream_words) & ~3u);
+      if (lane == 0 && nhi >= nlo && w1 > w0) bulk_prefetch_l2(p.stream + w0, (w1 - w0) * 4u);
+    }
     __syncwarp();
-    emit_groups<MODE>(p, stage, info, umask, c_first * cg, static_cast<int>(g_lo - c_first * cg),
+    emit_groups<MODE>(p, stage, info, c_first * cg, static_cast<int>(g_lo - c_first * cg),
                       static_cast<int>(g_hi - c_first * cg), og0, zero);
     __syncwarp();
   }
@@ -450,6 +570,7 @@ uw_status fill_params(const uw_matrix* m, void* out, uint32_t* status, DecodePar
   p.stream_words = m->L.stream_words;
   p.n_rows = m->L.rows;
   p.chunk_groups = m->L.chunk_groups;
+  p.cg_magic = (65536u + static_cast<uint32_t>(p.chunk_groups) - 1) / static_cast<uint32_t>(p.chunk_groups);
   p.gpr = static_cast<int32_t>(m->L.cols / 64);
   p.wpr = m->L.words_per_row;
   p.max_len = m->cb.max_len;
@@ -460,10 +581,11 @@ uw_status fill_params(const uw_matrix* m, void* out, uint32_t* status, DecodePar
   return UW_OK;
 }
 
-// Warps per block: the index stage (1 KB per chunk group per warp) and the
-// group info (128 bytes per chunk group per warp) within kStageBudget, at
-// most 8.
-int warps_per_block(int cg) { return std::max(1, std::min(8, kStageBudget / (cg * 1152))); }
+// Warps per block: as many warps' shared memory as fit in kBlockSmem, at
+// most kMaxWarps.
+int warps_per_block(int cg) {
+  return std::max(1, std::min(kMaxWarps, kBlockSmem / (warp_words(cg) * 4)));
+}
 
 // Per device: the kernel's shared-memory opt-in (set once: the call is not
 // free and may wait for the device) and its resident blocks per SM for each
@@ -480,8 +602,9 @@ uw_status resident_blocks(int dev, size_t smem, int threads, int* per_sm) {
     return UW_OK;
   }
   if (!attr_set[dev & 63]) {
+    // the largest request: one warp of the largest chunk size, or kBlockSmem
     if (cudaFuncSetAttribute(decode_kernel<MODE, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kStageBudget + 8 * kRowStreamWords * 4) != cudaSuccess)
+                             std::max(kBlockSmem, warp_words(16) * 4)) != cudaSuccess)
       return UW_ERR_CUDA;
     attr_set[dev & 63] = true;
   }
@@ -497,9 +620,8 @@ template <int MODE, bool ROWS>
 uw_status launch(const DecodeParams& p, const DeviceInfo& dev, cudaStream_t s) {
   if (p.n_items <= 0) return UW_OK;
   const int W = warps_per_block(p.chunk_groups);
-  // (also the table build's kLutSize-word scratch)
-  const size_t smem = std::max<size_t>(static_cast<size_t>(W) * p.chunk_groups * 1152, kLutSize * 2) +
-                      (ROWS ? static_cast<size_t>(W) * kRowStreamWords * 4 : 0);
+  // (also the table build's kLutSize-halfword scratch)
+  const size_t smem = std::max<size_t>(static_cast<size_t>(W) * warp_words(p.chunk_groups) * 4, kLutSize * 2);
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return UW_ERR_CUDA;
   int per_sm = 0;

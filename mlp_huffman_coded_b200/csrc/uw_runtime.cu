@@ -99,6 +99,8 @@ uw_status check_matrix(const uw_matrix* m) {
       L.n_verbatim < 0 || L.n_verbatim > L.n_groups)
     return UW_ERR_CORRUPT;
   if (m->cb.max_len > UW_MAX_CODE_LEN) return UW_ERR_CORRUPT;
+  for (int i = 0; i < UW_PALETTE; ++i)
+    if (m->cb.code_len[i] > m->cb.max_len) return UW_ERR_CORRUPT;  // the decoders index per-length tables
   if (!m->sm || !m->stream || !m->chunk_bit_off || !m->vflags || !m->vprefix) return UW_ERR_INVALID_ARG;
   if (L.n_verbatim > 0 && !m->verbatim) return UW_ERR_INVALID_ARG;
   if (!aligned16(m->sm) || !aligned16(m->stream) || !aligned16(m->chunk_bit_off) || !aligned16(m->vflags) ||

@@ -144,6 +144,25 @@ def test_size_query_and_argument_errors():
                          None) == uw.UW_ERR_CORRUPT
 
 
+
+def test_decoders_reject_a_code_length_above_max_len_on_the_host():
+    """The decoders index per-length tables by each code length: a codebook
+    whose code_len exceeds its own max_len is refused before any launch (the
+    pointers here are never dereferenced)."""
+    w = synth.weight_matrix(64, 256, 0.02, 0.0, 1.0, 5)
+    enc = uw.encode(w)
+    m = uw.Matrix()
+    m.L = enc.layout
+    m.cb = enc.cb
+    for f in ("sm", "stream", "chunk_bit_off", "vflags", "vprefix"):
+        setattr(m, f, 0x10000)
+    i = int(np.argmax(np.array(list(m.cb.code_len))))
+    m.cb.code_len[i] = m.cb.max_len + 1
+    lib = uw.lib()
+    for fn in (lib.uw_decode_full, lib.uw_decode_exponent_only, lib.uw_transcode_palette):
+        assert fn(C.byref(m), 0x20000, 0x30000, 256, None) == uw.UW_ERR_CORRUPT
+
+
 def test_workspace_bytes_is_host_only():
     w = synth.weight_matrix(256, 512, 0.02, 5e-4, 200.0, 0)
     enc = uw.encode(w)
