@@ -112,57 +112,83 @@ struct DecodeTables {
   uint32_t count[17];      // codes of each length
   uint32_t offset[17];     // index of the first symbol of each length
   uint8_t sorted[16];      // symbols in (length, index) order
+  // codes of at most 11 bits in that order: their first 11-bit prefix and
+  // symbol | length << 4
+  uint16_t start[16];
+  uint16_t short_ent[16];
+  uint32_t n_short;
+  uint16_t lut[kLutSize];  // build scratch: the first code of each prefix
 };
 
-// lut: kLutSize words of scratch (the first code of each prefix, sym |
+// Where the build scratch keeps the first code of 11-bit prefix x: bits 1..5
+// (the bank) XORed with bits 6..10, so that the consecutive prefixes of a
+// warp shifted left by a code length still fall on distinct banks.
+__device__ __forceinline__ uint32_t lut_slot(uint32_t x) { return x ^ ((x >> 5) & 0x3Eu); }
+
+// lut: kLutSize halfwords of scratch (the first code of each prefix, sym |
 // len << 4, len 0 = longer than the table), needed only while building.
 __device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables& t, uint16_t* lut) {
-  // warp 0: code counts per length, the canonical first codes, and the
-  // symbols in (length, index) order (each symbol placed at its rank in
-  // that order)
+  // warp 0: code counts per length (ballots), the canonical first code and
+  // first rank of each length (lane l holds length l's), and each symbol's
+  // rank in (length, index) order and canonical code
   if (threadIdx.x < 32) {
-    const int i = threadIdx.x;
-    const int li = i < 16 ? p.code_len[i] : 0;
-    if (i <= 16) t.count[i] = 0;
-    __syncwarp();
-    if (i < 16 && li > 0) {
-      int rank = 0;
-      for (int j = 0; j < 16; ++j) {
-        const int lj = p.code_len[j];
-        rank += (lj > 0 && (lj < li || (lj == li && j < i))) ? 1 : 0;
+    const uint32_t lane = threadIdx.x;
+    const uint32_t li = lane < 16 ? p.code_len[lane] : 0u;
+    uint32_t first_l = 0, offset_l = 0, count_l = 0;
+    uint32_t code = 0, pos = 0;
+#pragma unroll
+    for (uint32_t l = 1; l <= 16; ++l) {
+      const uint32_t cnt = __popc(__ballot_sync(0xffffffffu, li == l));
+      if (lane == l) {
+        first_l = code;
+        offset_l = pos;
+        count_l = cnt;
       }
-      t.sorted[rank] = static_cast<uint8_t>(i);
-      atomicAdd(&t.count[li], 1u);
+      code = (code + cnt) << 1;
+      pos += cnt;
     }
-    __syncwarp();
-    if (i == 0) {
-      uint32_t code = 0, pos = 0;
-      for (int l = 1; l <= 16; ++l) {
-        t.first[l] = code;
-        t.offset[l] = pos;
-        code = (code + t.count[l]) << 1;
-        pos += t.count[l];
+    if (lane >= 1 && lane <= 16) {
+      t.first[lane] = first_l;
+      t.offset[lane] = offset_l;
+      t.count[lane] = count_l;
+    }
+    const uint32_t same = __match_any_sync(0xffffffffu, li);
+    const uint32_t before = __popc(same & ((1u << lane) - 1u));  // lanes below with the same length
+    const uint32_t rank = __shfl_sync(0xffffffffu, offset_l, li & 31u) + before;
+    const uint32_t mine = __shfl_sync(0xffffffffu, first_l, li & 31u) + before;
+    if (lane < 16 && li > 0) {
+      t.sorted[rank] = static_cast<uint8_t>(lane);
+      if (li <= kLutBits) {
+        t.start[rank] = static_cast<uint16_t>(mine << (kLutBits - li));
+        t.short_ent[rank] = static_cast<uint16_t>(lane | (li << 4));
       }
+    }
+    const uint32_t n_short = __shfl_sync(0xffffffffu, offset_l, kLutBits + 1);
+    const uint32_t base = __shfl_sync(0xffffffffu, first_l, kLutBits) + __shfl_sync(0xffffffffu, count_l, kLutBits);
+    if (lane == 0) {
+      t.n_short = n_short;
+      t.long_base = base;  // end of the codes of <= 11 bits
     }
   }
   __syncthreads();
-  const int lim = p.max_len < kLutBits ? p.max_len : kLutBits;
-  for (int v = threadIdx.x; v < kLutSize; v += blockDim.x) {
-    uint16_t ent = 0;
-    for (int l = 1; l <= lim; ++l) {
-      const uint32_t code = static_cast<uint32_t>(v) >> (kLutBits - l);
-      const uint32_t d = code - t.first[l];
-      if (t.count[l] && d < t.count[l]) {
-        ent = static_cast<uint16_t>(t.sorted[t.offset[l] + d] | (l << 4));
-        break;
-      }
-    }
-    lut[v] = ent;
-  }
-  __syncthreads();
+  // the first code of every 11-bit prefix below long_base: the last short
+  // code whose start is at most the prefix (starts increase with the rank;
+  // ranks past n_short count as never started).  The starts go to registers
+  // once; the prefix x is stored at lut_slot(x).
   {
-    const uint32_t base = t.first[kLutBits] + t.count[kLutBits];  // end of the codes of <= 11 bits
-    if (threadIdx.x == 0) t.long_base = base;
+    const uint32_t n_short = t.n_short, base = t.long_base;
+    uint32_t s[16];
+#pragma unroll
+    for (uint32_t k = 0; k < 16; ++k) s[k] = k < n_short ? t.start[k] : 0xFFFFu;
+    for (int v = threadIdx.x; v < kLutSize; v += blockDim.x) {
+      uint32_t r = 0;
+#pragma unroll
+      for (uint32_t k = 1; k < 16; ++k) r += s[k] <= static_cast<uint32_t>(v) ? 1u : 0u;
+      lut[lut_slot(v)] = static_cast<uint32_t>(v) < base ? t.short_ent[r] : static_cast<uint16_t>(0);
+    }
+  }
+  {
+    const uint32_t base = t.long_base;
     for (int s = threadIdx.x; s < 17 * 16; s += blockDim.x) {
       const uint32_t row = static_cast<uint32_t>(s) >> 4;
       const uint32_t val = ((base + row) << 4) | (static_cast<uint32_t>(s) & 15u);  // 15-bit value
@@ -177,13 +203,14 @@ __device__ __forceinline__ void build_tables(const DecodeParams& p, DecodeTables
       t.sub[s] = ent;
     }
   }
+  __syncthreads();
   // chain single-code lookups inside the 11-bit prefix: a code shorter than
   // the bits left is decoded correctly whatever the zero padding (prefix-free)
   for (int v = threadIdx.x; v < kLutSize; v += blockDim.x) {
     uint32_t idx = 0, cum = 0;
     int used = 0, n = 0;
     while (n < 4 && used < kLutBits) {
-      const uint32_t e = lut[(static_cast<uint32_t>(v) << used) & (kLutSize - 1)];
+      const uint32_t e = lut[lut_slot((static_cast<uint32_t>(v) << used) & (kLutSize - 1))];
       const int l = (e >> 4) & 15;
       if (l == 0 || l > kLutBits - used) break;
       idx |= (e & 15u) << (4 * n);
@@ -465,7 +492,6 @@ template <int MODE, bool ROWS>
 __global__ void __launch_bounds__(32 * kMaxWarps, 1) decode_kernel(const DecodeParams p) {
   __shared__ DecodeTables t;
   extern __shared__ __align__(16) uint32_t dsm[];
-  build_tables(p, t, reinterpret_cast<uint16_t*>(dsm));  // the stage holds the build scratch
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int W = blockDim.x >> 5;
   const int cg = p.chunk_groups;
@@ -474,8 +500,28 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1) decode_kernel(const DecodeP
   uint32_t* sbuf = reinterpret_cast<uint32_t*>(info + 32 * cg);
   const int64_t cap = stream_cap_words(cg);
   const uint32_t last_word = static_cast<uint32_t>(p.stream_words - 1);
-  for (int64_t it = static_cast<int64_t>(blockIdx.x) * W + warp; it < p.n_items;
-       it += static_cast<int64_t>(gridDim.x) * W) {
+  const int64_t it0 = static_cast<int64_t>(blockIdx.x) * W + warp;
+  // The first item's chunk offsets and group sources are read, and its
+  // stream span is prefetched into L2, before the tables are built, so that
+  // their latency overlaps the build.
+  bool pre = false;
+  uint32_t pb0 = 0, pb1 = 0;
+  int pn = 0;
+  if (!ROWS && it0 < p.n_items) {
+    const int64_t cf = it0 * 32, ce = min(cf + 32, p.n_chunks), c = cf + lane;
+    const uint32_t lo = __ldg(p.off + cf), hi = __ldg(p.off + ce);
+    if (c < ce) {
+      pb0 = __ldg(p.off + c);
+      pb1 = __ldg(p.off + c + 1);
+    }
+    const uint32_t w0 = (lo >> 5) & ~3u;
+    const uint32_t w1 = min(((hi >> 5) + 6u) & ~3u, static_cast<uint32_t>(p.stream_words) & ~3u);
+    if (lane == 0 && hi >= lo && w1 > w0) bulk_prefetch_l2(p.stream + w0, (w1 - w0) * 4u);
+    if (c < ce) pn = group_sources(p, c, info + lane * cg);
+    pre = true;
+  }
+  build_tables(p, t, t.lut);
+  for (int64_t it = it0; it < p.n_items; it += static_cast<int64_t>(gridDim.x) * W) {
     int64_t c_first, c_end, g_lo, g_hi, og0;
     bool zero = false;
     if (!ROWS) {
@@ -518,13 +564,14 @@ __global__ void __launch_bounds__(32 * kMaxWarps, 1) decode_kernel(const DecodeP
       // group sources, then step 1: the stream words of chunks [c_first,
       // c_end) plus the window's two-word overrun, when they fit the warp's
       // buffer
-      uint32_t b0 = 0, b1 = 0;
-      int n_coded = 0;
-      if (c < c_end) {
+      uint32_t b0 = pb0, b1 = pb1;
+      int n_coded = pn;
+      if (!pre && c < c_end) {
         b0 = __ldg(p.off + c);
         b1 = __ldg(p.off + c + 1);
         n_coded = group_sources(p, c, info + lane * cg);
       }
+      pre = false;
       const uint32_t blo = __shfl_sync(0xffffffffu, b0, 0), bhi = __shfl_sync(0xffffffffu, b1, nc - 1);
       const uint32_t sbase = blo >> 5;
       const int64_t span = static_cast<int64_t>(bhi >> 5) + 3 - sbase;
@@ -620,8 +667,7 @@ template <int MODE, bool ROWS>
 uw_status launch(const DecodeParams& p, const DeviceInfo& dev, cudaStream_t s) {
   if (p.n_items <= 0) return UW_OK;
   const int W = warps_per_block(p.chunk_groups);
-  // (also the table build's kLutSize-halfword scratch)
-  const size_t smem = std::max<size_t>(static_cast<size_t>(W) * warp_words(p.chunk_groups) * 4, kLutSize * 2);
+  const size_t smem = static_cast<size_t>(W) * warp_words(p.chunk_groups) * 4;
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return UW_ERR_CUDA;
   int per_sm = 0;
