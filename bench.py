@@ -484,8 +484,8 @@ def run_gpu(args, world, rank, local):
 
 
 def run_gemm_case(args, local):
-    """One matrix (gate, 14336x4096) through one pipeline: the unit the ncu
-    profiles in profiles/ are taken on.  Prints a small JSON line."""
+    """One matrix (gate, 14336x4096) through one pipeline: the unit that ncu
+    captures of the GEMM are taken on.  Prints a small JSON line."""
     import torch
     from mlp_huffman_coded_b200 import synth, uw
     torch.cuda.set_device(local)
