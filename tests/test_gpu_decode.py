@@ -99,6 +99,49 @@ def test_long_codes_use_the_slow_path():
     _check(w)
 
 
+def _flat_exponents(rows, cols, seed):
+    """Exponents drawn evenly from 16 values: every code is 4 bits long."""
+    rng = np.random.default_rng(seed)
+    exp = rng.integers(110, 126, (rows, cols)).astype(np.uint16)
+    return ((rng.integers(0, 2, exp.shape).astype(np.uint16) << 15) | (exp << 7)
+            | rng.integers(0, 128, exp.shape).astype(np.uint16)).astype(np.uint16)
+
+
+@pytest.mark.parametrize("chunk_groups", [1, 4, 16])
+def test_wide_codes_read_the_stream_from_global_memory(chunk_groups):
+    # 4-bit codes: the stream words of a warp's 32 chunks (256 * chunk_groups
+    # words) outgrow its shared-memory copy, so the lanes read the stream
+    # from global memory instead
+    w = _flat_exponents(96, 2048, 12)
+    assert set(uw.encode(w, chunk_groups=chunk_groups).cb.code_len) == {4}
+    _check(w, chunk_groups)
+
+
+def test_warps_mixing_staged_and_global_streams():
+    # rows alternate between 4-bit codes and the usual ~2.6-bit ones, so
+    # neighbouring warps take different stream paths in one launch
+    a = _flat_exponents(64, 2048, 13)
+    b = synth.weight_matrix(64, 2048, 0.02, 1e-4, 100.0, 14)
+    w = np.empty((128, 2048), np.uint16)
+    w[0::2], w[1::2] = a, b
+    for cg in (1, 4):
+        _check(w, cg)
+
+
+def test_invalid_codes_of_an_incomplete_code_are_reported():
+    # a one-symbol code ("0"): every 1 bit in the stream is an invalid code
+    w = np.full((64, 1024), 120 << 7, dtype=np.uint16)
+    enc = uw.encode(w)
+    assert enc.cb.n_symbols == 1
+    enc.stream[:-2] = np.uint32(0xFFFFFFFF)
+    dm = uw.DeviceMatrix(enc)
+    ws = uw.Workspace(256)
+    import torch
+    out = torch.empty(64 * 1024 // 2, dtype=torch.uint8, device="cuda")
+    uw.transcode_palette(dm, out, ws)
+    assert ws.status() == uw.UW_ERR_CORRUPT
+
+
 def test_full_size_gate_matrix_bit_exact():
     p = synth.WORKLOADS["gate_14336x4096"]
     w = synth.weight_matrix(p["rows"], p["cols"], p["sigma"], p["outlier_rate"], p["outlier_scale"], p["seed"])
