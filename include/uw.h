@@ -323,7 +323,10 @@ UW_API uw_status uw_encode_gpu(const uint16_t* w, int64_t rows, int64_t cols, co
  * original word bit for bit, verbatim groups copied from the verbatim store.
  * Reads sm + stream + offsets + flags + verbatim; writes 2 bytes per
  * element.  Errors: UW_ERR_INVALID_ARG (NULL or misaligned pointers),
- * UW_ERR_WORKSPACE_TOO_SMALL (< 256 bytes), UW_ERR_NO_DEVICE, UW_ERR_CUDA;
+ * UW_ERR_WORKSPACE_TOO_SMALL (< 256 bytes), UW_ERR_UNSUPPORTED_SHAPE /
+ * UW_ERR_CORRUPT (a layout whose sizes disagree with rows and cols, or a
+ * codebook with max_len > 15 or a code length above max_len; found on the
+ * host, nothing is launched), UW_ERR_NO_DEVICE, UW_ERR_CUDA;
  * on the device, a chunk whose code lengths do not end exactly at the next
  * chunk's offset (or an invalid code) records UW_ERR_CORRUPT in the status
  * word, and every read stays inside the stream. */
